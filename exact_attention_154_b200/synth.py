@@ -1,0 +1,153 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module holds no attention arithmetic: it only draws the inputs (and the
+sampled query rows used to check large shapes), so that the CUDA path and the
+CPU oracle see exactly the same values.
+
+Recipe: a CPU ``torch.Generator`` seeded with the workload's seed draws
+``randn`` in fp32, the values are multiplied by the workload's standard
+deviation and rounded once to the compute dtype.  The oracle widens those
+rounded values to fp64, so both sides start from identical numbers.
+
+The workloads follow the shapes the pages use: the single-head ``[B, N, d]``
+layout of ``flash_attention_forward`` in "flash_attention.py"
+(forceinjection.github.io); the packed ``qkv`` call of section 5.2 of
+"Windows下RTX 3090编译Flash Attention 2.8.3全指南" (intelliparadigm.com); the
+GPT-3-like head count of section 1.2 of "2.3 FlashAttention与IO感知注意力(1)"
+(aiknowledge.cn); the sequence-length list of the A100 table of
+"flash-attention与TensorRT 10集成" (blog.gitcode.com); and head dim 256, the
+largest that page lists.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+FP16, BF16 = 0, 1
+TORCH_DTYPE = {FP16: torch.float16, BF16: torch.bfloat16}
+DTYPE_NAME = {FP16: "f16", BF16: "bf16"}
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One attention forward problem.
+
+    ``layout`` is ``"bhnd"`` (separate q, k, v of shape [B, H, N, d]) or
+    ``"packed"`` (one qkv of shape [B, N, 3, H, d]).
+    """
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    dtype: int
+    causal: bool
+    seed: int
+    layout: str = "bhnd"
+    sigma_qk: float = 1.0
+    sigma_v: float = 1.0
+    extra: dict = field(default_factory=dict, compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def flops(self) -> float:
+        """4*B*H*N^2*d, halved for the causal mask."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def describe(self) -> dict:
+        return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N,
+                "d": self.d, "dtype": DTYPE_NAME[self.dtype],
+                "causal": self.causal, "layout": self.layout, "seed": self.seed}
+
+
+def single_head_n256() -> Workload:
+    return Workload("single-head fwd [1,256,64] fp16 non-causal", 1, 1, 256, 64,
+                    FP16, False, 42)
+
+
+def packed_qkv_b2_n256_h12() -> Workload:
+    return Workload("packed-qkv fwd [2,256,3,12,64] fp16 non-causal", 2, 12, 256, 64,
+                    FP16, False, 43, layout="packed")
+
+
+def many_heads_causal_n2048() -> Workload:
+    return Workload("causal fwd [1,128,2048,128] bf16", 1, 128, 2048, 128, BF16,
+                    True, 44)
+
+
+SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384)
+
+
+def seqlen_sweep(N: int, causal: bool) -> Workload:
+    if N not in SWEEP_N:
+        raise ValueError(f"N must be one of {SWEEP_N}")
+    seed = 45 + int(round(math.log2(N // 512)))
+    tag = "causal" if causal else "non-causal"
+    return Workload(f"seqlen sweep fwd B={16384 // N},H=16,N={N},d=128 bf16 {tag}",
+                    16384 // N, 16, N, 128, BF16, causal, seed)
+
+
+def headdim256_causal() -> Workload:
+    return Workload("head-dim 256 causal fwd [1,8,8192,256] bf16, q,k ~ N(0,3^2)",
+                    1, 8, 8192, 256, BF16, True, 50, sigma_qk=3.0)
+
+
+def all_workloads() -> list[Workload]:
+    w = [single_head_n256(), packed_qkv_b2_n256_h12(), many_heads_causal_n2048()]
+    for n in SWEEP_N:
+        for c in (False, True):
+            w.append(seqlen_sweep(n, c))
+    w.append(headdim256_causal())
+    return w
+
+
+def make_inputs(w: Workload):
+    """CPU tensors in the compute dtype.
+
+    ``bhnd`` -> ``(q, k, v)`` each [B, H, N, d]; ``packed`` -> ``(qkv,)`` of
+    shape [B, N, 3, H, d] (index 0/1/2 of axis 2 = q/k/v).
+    """
+    g = torch.Generator().manual_seed(w.seed)
+    dt = TORCH_DTYPE[w.dtype]
+    if w.layout == "packed":
+        qkv = torch.randn((w.B, w.N, 3, w.H, w.d), generator=g, dtype=torch.float32)
+        qkv[:, :, 0:2] *= w.sigma_qk
+        qkv[:, :, 2] *= w.sigma_v
+        return (qkv.to(dt),)
+    shape = (w.B, w.H, w.N, w.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32) * w.sigma_qk
+    k = torch.randn(shape, generator=g, dtype=torch.float32) * w.sigma_qk
+    v = torch.randn(shape, generator=g, dtype=torch.float32) * w.sigma_v
+    return q.to(dt), k.to(dt), v.to(dt)
+
+
+def unpack_qkv(qkv: torch.Tensor):
+    """[B, N, 3, H, d] -> three [B, H, N, d] tensors (a pure re-indexing)."""
+    return tuple(qkv[:, :, i].permute(0, 2, 1, 3).contiguous() for i in range(3))
+
+
+def sample_rows(N: int, seed: int, count: int = 512) -> np.ndarray:
+    """Sorted query rows to check at large N: ``count`` distinct rows drawn with
+    ``numpy.random.default_rng(seed + 1000)``, always including 0, 127, 128 and
+    N-1 (when they exist).  Every row is independent of the others given K and
+    V, so a sample checks the rows it names exactly."""
+    must = {r for r in (0, 127, 128, N - 1) if 0 <= r < N}
+    if N <= count:
+        return np.arange(N, dtype=np.int32)
+    rng = np.random.default_rng(seed + 1000)
+    pick = rng.choice(N, size=count, replace=False)
+    return np.array(sorted(must.union(int(x) for x in pick)), dtype=np.int32)
+
+
+def random_inputs(B, H, N, d, dtype, seed, sigma_qk=1.0, sigma_v=1.0):
+    """[B, H, N, d] q, k, v for ad-hoc test shapes (same recipe)."""
+    w = Workload("adhoc", B, H, N, d, dtype, False, seed, sigma_qk=sigma_qk,
+                 sigma_v=sigma_v)
+    return make_inputs(w)

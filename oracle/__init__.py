@@ -1,0 +1,146 @@
+"""fp64 CPU oracle for the exact attention forward.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` are the only callers.  Nothing in the product
+package imports this module, and this module imports nothing from it.
+
+Three independent implementations live here:
+
+* :func:`attention` -- the plain definition (scores, row max, exp, sum, P V,
+  logsumexp) in C with OpenMP over rows, fp64 throughout
+  (``fa_oracle.c``).  Follows the standard attention of
+  "2.3 FlashAttention与IO感知注意力(1)" (aiknowledge.cn), section 1.1, and the
+  ``standard_attention`` function of "flash_attention.py"
+  (forceinjection.github.io).
+* :func:`oracle.tiled.flash_forward` -- the tiled online-softmax recurrence of
+  ``flash_attention_forward`` in the same file, restated in NumPy fp64 and
+  extended with the causal mask and the logsumexp output.
+* :func:`oracle.brute.attention_fsum` -- a scalar pure-Python version using
+  ``math.fsum`` for tiny inputs.
+
+Parity status: every function here is pinned by tests in
+``tests/test_oracle_pins.py`` (closed forms, invariants, brute force and the
+recurrence-equals-definition check); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libfa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``fa_oracle.c`` into ``libfa_oracle.so`` next to it (gcc, OpenMP).
+
+    Plain ``-O2`` with no fast-math flags, so every operation is IEEE fp64.
+    """
+    if not force and os.path.exists(_LIB_PATH) and (
+        os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)
+    ):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c99",
+           "-fno-fast-math", "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            dp = ctypes.POINTER(ctypes.c_double)
+            ip = ctypes.POINTER(ctypes.c_int)
+            lib.oracle_attention_fwd.argtypes = [
+                dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int, ip, ctypes.c_int]
+            lib.oracle_attention_fwd.restype = ctypes.c_int
+            lib.oracle_attention_probs.argtypes = [
+                dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                ctypes.c_int, dp]
+            lib.oracle_attention_probs.restype = ctypes.c_int
+            lib.oracle_num_threads.argtypes = []
+            lib.oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _as_f64(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # a torch tensor (CPU); widening fp16/bf16 is exact
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _dptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle runs with (``OMP_NUM_THREADS`` or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def attention(q, k, v, scale: float | None = None, causal: bool = False,
+              rows=None):
+    """Exact attention forward in fp64.
+
+    ``q, k, v``: ``[B, H, N, d]`` (or ``[N, d]`` / ``[B, N, d]``, treated as
+    H=1 / B=1) arrays or CPU tensors.  ``scale=None`` means ``1/sqrt(d)``.
+    ``rows``: optional sequence of query indices; the result then holds only
+    those rows, in that order, for every (b, h).
+
+    Returns ``(O, LSE)`` with ``O`` shaped like ``q`` restricted to ``rows`` and
+    ``LSE`` shaped ``q.shape[:-1]`` restricted likewise (natural log).
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    lead = q.shape[:-2]
+    N, d = q.shape[-2], q.shape[-1]
+    if q.ndim == 2:
+        B, H = 1, 1
+    elif q.ndim == 3:
+        B, H = q.shape[0], 1
+    elif q.ndim == 4:
+        B, H = q.shape[0], q.shape[1]
+    else:
+        raise ValueError("expected 2-D, 3-D or 4-D inputs")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    rows_arr = np.arange(N, dtype=np.int32) if rows is None else np.ascontiguousarray(
+        np.asarray(rows, dtype=np.int32))
+    nr = int(rows_arr.size)
+    o = np.empty((B, H, nr, d), dtype=np.float64)
+    lse = np.empty((B, H, nr), dtype=np.float64)
+    rc = _load().oracle_attention_fwd(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(o), _dptr(lse), B, H, N, d,
+        float(scale), int(bool(causal)),
+        rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), nr)
+    if rc != 0:
+        raise ValueError(f"oracle_attention_fwd failed ({rc})")
+    return o.reshape(lead + (nr, d)), lse.reshape(lead + (nr,))
+
+
+def probs(q, k, i: int, scale: float | None = None, causal: bool = False):
+    """Normalised attention weights of query row ``i`` for one ``[N, d]`` slice."""
+    q, k = _as_f64(q), _as_f64(k)
+    N, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    p = np.empty(N, dtype=np.float64)
+    rc = _load().oracle_attention_probs(_dptr(q), _dptr(k), N, d, float(scale),
+                                        int(bool(causal)), int(i), _dptr(p))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_probs failed ({rc})")
+    return p
