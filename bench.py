@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 exact attention forward.
+
+One step = one attention forward (one kernel launch) over the whole workload,
+inputs resident in HBM.  Default workload: the sequence-length sweep point
+N=4096, B=4, H=16, d=128, bf16, non-causal -- the smallest N at which the
+throughput target (>= 60% of the dense bf16 tensor-core peak) applies.
+FLOPs per step = 4*B*H*N^2*d (halved when causal).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+  python bench.py --sweep                 # one JSON line per benchmark workload
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own copy of
+the workload (independent (b, h) problems, no collective on the data path:
+weak scaling); the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_attention_154_b200 import fa, synth  # noqa: E402
+
+METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense tensor-core peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fa_fwd_sm100_traffic.md")
+KERNEL_SOURCES = ["exact_attention_154_b200/csrc/fa_fwd_sm100.cuh",
+                  "exact_attention_154_b200/csrc/sm100_ptx.cuh",
+                  "exact_attention_154_b200/csrc/fa_api.cu"]
+
+
+def workloads_by_key():
+    table = {
+        "single-head-n256": synth.single_head_n256(),
+        "packed-b2-n256-h12": synth.packed_qkv_b2_n256_h12(),
+        "causal-h128-n2048": synth.many_heads_causal_n2048(),
+        "hd256-causal-n8192": synth.headdim256_causal(),
+    }
+    for n in synth.SWEEP_N:
+        table[f"sweep-n{n}"] = synth.seqlen_sweep(n, False)
+        table[f"sweep-n{n}-causal"] = synth.seqlen_sweep(n, True)
+    return table
+
+
+DEFAULT_WORKLOAD = "sweep-n4096"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source and this workload; else None."""
+    try:
+        text = open(PROFILE_TRAFFIC).read()
+    except OSError:
+        return None
+    src = re.search(r"source_sha256:\s*([0-9a-f]+)", text)
+    if not src or src.group(1) != kernel_source_hash():
+        return None
+    m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload_key)}\]:\s*([0-9.eE+]+)", text)
+    return float(m.group(1)) if m else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        # samples under load: the upper half of the SM clocks seen
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def device_inputs(w):
+    if w.layout == "packed":
+        (qkv,) = synth.make_inputs(w)
+        return (qkv.cuda(),)
+    return tuple(t.cuda() for t in synth.make_inputs(w))
+
+
+def launcher(w, dev_inputs):
+    """Returns a zero-argument callable issuing one forward on the current stream."""
+    if w.layout == "packed":
+        (qkv,) = dev_inputs
+        out = torch.empty((w.B, w.N, w.H, w.d), device="cuda", dtype=qkv.dtype)
+        lse = torch.empty((w.B, w.H, w.N), device="cuda", dtype=torch.float32)
+        lib = fa.load()
+        args = (qkv.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B, w.N, w.H, w.d, 0.0,
+                int(w.causal), 0.0, w.dtype)
+
+        def go():
+            rc = lib.fa_fwd_qkvpacked(*args, torch.cuda.current_stream().cuda_stream)
+            if rc:
+                raise fa.FaError(rc, "fa_fwd_qkvpacked")
+        return go, (out, lse)
+    q, k, v = dev_inputs
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), device="cuda", dtype=torch.float32)
+    lib = fa.load()
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B, w.H,
+            w.N, w.d, 0.0, int(w.causal), w.dtype)
+
+    def go():
+        rc = lib.fa_fwd(*args, torch.cuda.current_stream().cuda_stream)
+        if rc:
+            raise fa.FaError(rc, "fa_fwd")
+    return go, (out, lse)
+
+
+def time_device(go, steps, warmup, world):
+    for _ in range(warmup):
+        go()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        go()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    ms = start.elapsed_time(end) / steps
+    return dist_max(ms, world)
+
+
+def time_e2e(w, steps, warmup, world):
+    """Same metric through the public Python API with pinned host inputs:
+    H2D of q, k, v (or qkv), the forward, D2H of O and LSE, every step."""
+    host = [t.pin_memory() for t in synth.make_inputs(w)]
+    dev = [torch.empty_like(t, device="cuda") for t in host]
+    if w.layout == "packed":
+        o_host = torch.empty((w.B, w.N, w.H, w.d), dtype=host[0].dtype).pin_memory()
+    else:
+        o_host = torch.empty_like(host[0]).pin_memory()
+    lse_host = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for h, d in zip(host, dev):
+            d.copy_(h, non_blocking=True)
+        if w.layout == "packed":
+            o, lse = fa.fwd_qkvpacked(dev[0], causal=w.causal)
+        else:
+            o, lse = fa.fwd(dev[0], dev[1], dev[2], causal=w.causal)
+        o_host.copy_(o, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    ms = dist_max(start.elapsed_time(end) / steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * 4
+    return ms, h2d, d2h
+
+
+def row_flops(w, rows):
+    """Algorithmic FLOPs of the given query rows (4*d per visible key)."""
+    if w.causal:
+        return float(sum(4.0 * w.d * (int(r) + 1) for r in rows))
+    return 4.0 * w.d * w.N * len(rows)
+
+
+def cpu_oracle_sample(w, target_s=12.0, max_rows_per_head=None):
+    """Times the fp64 oracle, as it stands, on a bounded sample of the
+    workload's query rows (the same rows in every (b, h)), on all host cores."""
+    import oracle
+    oracle.build()
+    if w.layout == "packed":
+        q, k, v = synth.unpack_qkv(synth.make_inputs(w)[0])
+    else:
+        q, k, v = synth.make_inputs(w)
+    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
+    rng = np.random.default_rng(w.seed + 2000)
+    sc = fa.default_scale(w.d)
+
+    def run(nrows):
+        rows = np.sort(rng.choice(w.N, size=nrows, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.attention(q64, k64, v64, scale=sc, causal=w.causal, rows=rows)
+        return time.perf_counter() - t0, row_flops(w, rows) * w.B * w.H, nrows
+
+    nrows = min(w.N, 4)
+    dt, fl, _ = run(nrows)
+    # grow the sample to about target_s seconds of CPU work
+    want = int(nrows * max(1.0, target_s / max(dt, 1e-3)))
+    cap = w.N if max_rows_per_head is None else min(w.N, max_rows_per_head)
+    nrows = max(1, min(cap, want))
+    dt, fl, nrows = run(nrows)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"{nrows} seeded query rows in each of the {w.B * w.H} (b, h) heads of "
+                      f"the workload (of N={w.N}), fp64 oracle, all host threads"}
+
+
+def clocks_ok(c):
+    bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+    return not (bad & set(c.get("reasons", [])))
+
+
+def bench_gpu(args, w, key, world, rank, local):
+    dev_in = device_inputs(w)
+    go, _ = launcher(w, dev_in)
+    flops = w.flops
+    steps = args.steps
+    with ClockSampler(local) as clk:
+        ms = time_device(go, steps, args.warmup, world)
+    clocks = clk.summary()
+    e2e_steps = max(3, min(steps, 50))
+    e2e_ms, h2d, d2h = time_e2e(w, e2e_steps, min(args.warmup, 3), world)
+    rc, detail = fa.device_status(clear=True)
+    if rc != fa.FA_OK:
+        raise RuntimeError(f"kernel watchdog fired ({detail:#x})")
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    value = world * flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": synth.DTYPE_NAME[w.dtype], "data": "synthetic (seeded randn, see DESIGN.md)",
+        "config": dict(w.describe(), workload_key=key,
+                       parallelism=f"replicas{world}" if world > 1 else "single-gpu",
+                       global_batch=w.B * world, seq_len=w.N,
+                       l2="inputs larger than L2 (q,k,v,o = %d MiB per step)" %
+                          ((4 if w.layout != "packed" else 0) * w.B * w.H * w.N * w.d * 2 >> 20)),
+        "pct_of_peak": {
+            "measured_burst": round(100 * achieved / peaks["bf16_tflops"], 2),
+            "measured_sustained": round(100 * achieved / peaks["bf16_tflops_sustained"], 2),
+            "nvidia_dense_bf16_datasheet_2250": round(100 * achieved / 2250.0, 2),
+            "peaks_source": peak_src},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peaks["bf16_tflops"], "unit": UNIT,
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak_note": f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json)"
+                                  if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+                     "traffic": profiled_traffic(key),
+                     "algorithmic_bytes": algorithmic_bytes(w),
+                     "kernel": "fa_fwd_kernel", "launches_per_step": 1},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps},
+        "gpu_launches": steps,
+        "clocks": clocks,
+    }
+    if not clocks_ok(clocks):
+        line["clocks_rejected"] = True
+    return line
+
+
+def algorithmic_bytes(w):
+    e = 2
+    return 4 * w.B * w.H * w.N * w.d * e + 4 * w.B * w.H * w.N
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads_by_key()))
+    ap.add_argument("--sweep", action="store_true", help="one line per benchmark workload")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    table = workloads_by_key()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        w = table[args.workload]
+        per_step = []
+        info = None
+        for _ in range(args.warmup if args.warmup < 1 else 0):
+            pass
+        budget = max(2.0, 120.0 / max(1, args.steps + 1))
+        for _ in range(args.steps):
+            info = cpu_oracle_sample(w, target_s=min(budget, 10.0))
+            per_step.append(info["value"])
+        value = statistics.median(per_step)
+        line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic (seeded randn)",
+                "config": dict(w.describe(), workload_key=args.workload),
+                "cpu_baseline": dict(info, value=round(value, 6)),
+                "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "gpu_launches": 0}
+        print(json.dumps(line))
+        return 0
+
+    world, rank, local = dist_setup()
+    keys = list(table) if args.sweep else [args.workload]
+    for key in keys:
+        w = table[key]
+        line = bench_gpu(args, w, key, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.sweep:
+            line["cpu_baseline"] = cpu_oracle_sample(w)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        torch.cuda.empty_cache()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,266 @@
+// fa_api.cu -- host side of libfa_sm100.so: argument checks, TMA tensor maps,
+// kernel selection by head dim / dtype, persistent-grid launch on the
+// caller's stream.  The C ABI is declared in include/fa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_fwd_sm100.cuh"
+
+namespace {
+
+using namespace fa_sm100;
+
+constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per mbarrier wait
+constexpr int kMaxDevices = 64;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mutex;
+EncodeTiledFn g_encode = nullptr;
+struct DeviceState {
+  bool ready = false;
+  bool is_sm100 = false;
+  int sm_count = 0;
+  bool attr_set[6] = {false, false, false, false, false, false};
+};
+DeviceState g_dev[kMaxDevices];
+
+int get_encode_fn() {
+  if (g_encode) return FA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                       &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  return FA_OK;
+}
+
+int device_state(DeviceState** out, int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    st.is_sm100 = (major == 10 && minor == 0);
+    st.sm_count = sms;
+    st.ready = true;
+  }
+  if (!st.is_sm100) return FA_ERR_DEVICE;
+  *out = &st;
+  *dev_out = dev;
+  return FA_OK;
+}
+
+// 4-D view (d, N, H, B) of one operand with element strides (1, sn, sh, sb);
+// box of 64 elements (128 bytes) x 128 rows, 128-byte swizzle, zero fill.
+int encode_operand(CUtensorMap* map, const void* ptr, int dtype, int d, int N, int H, int B,
+                   long long sn, long long sh, long long sb) {
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)sn * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType t =
+      dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = g_encode(map, t, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Kernel configuration per head dim: (Q tiles per work tile, K/V ring stages).
+template <int HD> struct Pick;
+template <> struct Pick<64> { static constexpr int QS = 2, KVS = 8; };
+template <> struct Pick<128> { static constexpr int QS = 2, KVS = 4; };
+template <> struct Pick<256> { static constexpr int QS = 1, KVS = 2; };
+
+int q_tiles_for(int d) { return d == 256 ? 1 : 2; }
+
+template <int HD, bool BF16>
+int launch(FwdParams& p, DeviceState& st, cudaStream_t stream) {
+  constexpr int QS = Pick<HD>::QS, KVS = Pick<HD>::KVS;
+  using C = FwdCfg<HD, QS, KVS, BF16>;
+  auto kernel = fa_fwd_kernel<HD, QS, KVS, BF16>;
+  const int slot = (HD == 64 ? 0 : HD == 128 ? 2 : 4) + (BF16 ? 1 : 0);
+  if (!st.attr_set[slot]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    st.attr_set[slot] = true;
+  }
+  const int grid = p.num_tiles < st.sm_count ? p.num_tiles : st.sm_count;
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int d, float* scale, int causal, int dtype) {
+  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_ARG;
+  if (!std::isfinite(*scale) || *scale < 0.f) return FA_ERR_ARG;
+  if (*scale == 0.f) *scale = 1.0f / std::sqrt(static_cast<float>(d));
+  // element counts and the tile count must fit the index types used on the device
+  const long long elems = (long long)B * H * N * d;
+  if (elems / d / N / H != B || elems > (1ll << 46)) return FA_ERR_ARG;
+  const long long qblocks = (N + 128LL * q_tiles_for(d) - 1) / (128LL * q_tiles_for(d));
+  if ((long long)B * H * qblocks > 0x7fffffffLL) return FA_ERR_ARG;
+  return FA_OK;
+}
+
+int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+        int d, float scale, int causal, int dtype, long long sn, long long sh, long long sb,
+        long long osn, long long osh, long long osb, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int rc = get_encode_fn();
+  if (rc != FA_OK) return rc;
+  DeviceState* st = nullptr;
+  int dev = 0;
+  if ((rc = device_state(&st, &dev)) != FA_OK) return rc;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  if ((rc = encode_operand(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb)) != FA_OK) return rc;
+  p.o = o;
+  p.lse = lse;
+  p.o_stride_n = osn;
+  p.o_stride_h = osh;
+  p.o_stride_b = osb;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int rows_per_tile = 128 * q_tiles_for(d);
+  p.num_qblocks = (N + rows_per_tile - 1) / rows_per_tile;
+  p.num_tiles = B * H * p.num_qblocks;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  const bool bf16 = dtype == FA_BF16;
+  switch (d) {
+    case 64: return bf16 ? launch<64, true>(p, *st, stream) : launch<64, false>(p, *st, stream);
+    case 128: return bf16 ? launch<128, true>(p, *st, stream) : launch<128, false>(p, *st, stream);
+    default: return bf16 ? launch<256, true>(p, *st, stream) : launch<256, false>(p, *st, stream);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, float scale, int causal, int dtype, struct CUstream_st* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_ARG;
+  int rc = check_common(B, H, N, d, &scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return FA_ERR_ALIGN;
+  const long long sn = d, sh = (long long)N * d, sb = (long long)H * N * d;
+  return run(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, sn, sh, sb, sn, sh, sb,
+             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int N, int H, int d, float scale,
+                     int causal, float dropout_p, int dtype, struct CUstream_st* stream) {
+  if (!qkv || !o) return FA_ERR_ARG;
+  if (!(dropout_p == 0.0f)) return std::isnan(dropout_p) ? FA_ERR_ARG : FA_ERR_UNSUPPORTED;
+  int rc = check_common(B, H, N, d, &scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(qkv) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return FA_ERR_ALIGN;
+  // qkv [B, N, 3, H, d]: q/k/v differ by H*d elements; o is [B, N, H, d].
+  const char* base = static_cast<const char*>(qkv);
+  const long long hd = (long long)H * d;
+  const long long sn = 3 * hd, sh = d, sb = (long long)N * 3 * hd;
+  return run(base, base + 2 * hd, base + 4 * hd, o, lse, B, H, N, d, scale, causal, dtype, sn, sh,
+             sb, hd, d, (long long)N * hd, reinterpret_cast<cudaStream_t>(stream));
+}
+
+const char* fa_strerror(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_ARG: return "invalid argument";
+    case FA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FA_ERR_HEADDIM: return "head dim must be 64, 128 or 256";
+    case FA_ERR_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
+    case FA_ERR_UNSUPPORTED: return "unsupported option (dropout_p must be 0)";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "kernel gave up on a bounded wait";
+    case FA_ERR_DEVICE: return "current device is not sm_100";
+    default: return "unknown status";
+  }
+}
+
+int fa_device_status(int clear, unsigned int* detail) {
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_fa_watchdog, sizeof(word)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_watchdog, &zero, sizeof(zero)) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+  }
+  if (detail) *detail = word;
+  return word ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st* stream) {
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return FA_ERR_ARG;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_launch_ctas(int B, int H, int N, int d, int causal) {
+  float scale = 0.f;
+  int rc = check_common(B, H, N, d, &scale, causal, FA_BF16);
+  if (rc != FA_OK) return rc;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState* st = nullptr;
+  int dev = 0;
+  if ((rc = device_state(&st, &dev)) != FA_OK) return rc;
+  const long long rows = 128LL * q_tiles_for(d);
+  const long long tiles = (long long)B * H * ((N + rows - 1) / rows);
+  return (int)(tiles < st->sm_count ? tiles : st->sm_count);
+}
+
+int fa_version(void) { return kVersion; }
+
+}  // extern "C"

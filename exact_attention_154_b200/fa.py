@@ -1,0 +1,177 @@
+"""Python binding of ``libfa_sm100.so`` (the C ABI in ``include/fa.h``).
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream; every step of the attention forward runs in the library's kernel.
+There is no fallback: if the library is missing or the device is not an
+sm_100 GPU, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+from .synth import BF16, FP16
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_sm100.so")
+_lock = threading.Lock()
+_lib = None
+
+FA_OK = 0
+FA_ERR_ARG, FA_ERR_ALIGN, FA_ERR_HEADDIM, FA_ERR_DTYPE = -1, -2, -3, -4
+FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_DEVICE = -5, -6, -7, -8
+
+#: every function the C header declares, with (restype, argtypes)
+_VP, _FP, _I, _F = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "fa_fwd_qkvpacked": (_I, [_VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
+    "fa_strerror": (ctypes.c_char_p, [_I]),
+    "fa_device_status": (_I, [_I, ctypes.POINTER(ctypes.c_uint)]),
+    "fa_debug_watchdog_selftest": (_I, [ctypes.c_ulonglong, _VP]),
+    "fa_launch_ctas": (_I, [_I, _I, _I, _I, _I]),
+    "fa_version": (_I, []),
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {strerror(status)} ({status})")
+        self.status = status
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -c 'import __graft_entry__ as g; g.build()'`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return load().fa_strerror(int(status)).decode()
+
+
+def version() -> int:
+    return int(load().fa_version())
+
+
+_DT = {torch.float16: FP16, torch.bfloat16: BF16}
+
+
+def _stream_ptr(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _check_tensor(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in _DT:
+        raise ValueError(f"{name} must be float16 or bfloat16")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
+        causal: bool = False, out: torch.Tensor | None = None,
+        lse: torch.Tensor | None = None, return_lse: bool = True):
+    """Attention forward on ``[B, H, N, d]`` tensors (``[B, N, d]`` is taken as H=1).
+
+    Returns ``(O, LSE)`` (``LSE`` is ``[B, H, N]`` fp32, or None when
+    ``return_lse`` is False).  ``scale=None`` means ``1/sqrt(d)``.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(t, name)
+    if not (q.shape == k.shape == v.shape) or q.dtype != k.dtype or q.dtype != v.dtype:
+        raise ValueError("q, k, v must share shape and dtype")
+    if q.dim() == 3:
+        B, N, d = q.shape
+        H = 1
+    elif q.dim() == 4:
+        B, H, N, d = q.shape
+    else:
+        raise ValueError("expected [B, H, N, d] or [B, N, d]")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_tensor(out, "out")
+        if out.shape != q.shape or out.dtype != q.dtype:
+            raise ValueError("out must match q")
+    lse_ptr = None
+    if return_lse:
+        if lse is None:
+            lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+        elif lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+            raise ValueError("lse must be a contiguous [B, H, N] float32 tensor")
+        lse_ptr = lse.data_ptr()
+    else:
+        lse = None
+    rc = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                       B, H, N, d, 0.0 if scale is None else float(scale), int(bool(causal)),
+                       _DT[q.dtype], _stream_ptr(q))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+    return out, lse
+
+
+def fwd_qkvpacked(qkv: torch.Tensor, dropout_p: float = 0.0, softmax_scale: float | None = None,
+                  causal: bool = False, out: torch.Tensor | None = None,
+                  return_lse: bool = True):
+    """Packed forward: ``qkv`` is ``[B, N, 3, H, d]``; returns ``(O [B, N, H, d], LSE [B, H, N])``."""
+    _check_tensor(qkv, "qkv")
+    if qkv.dim() != 5 or qkv.shape[2] != 3:
+        raise ValueError("qkv must be [B, N, 3, H, d]")
+    B, N, _, H, d = qkv.shape
+    if out is None:
+        out = torch.empty((B, N, H, d), device=qkv.device, dtype=qkv.dtype)
+    else:
+        _check_tensor(out, "out")
+    lse = torch.empty((B, H, N), device=qkv.device, dtype=torch.float32) if return_lse else None
+    rc = load().fa_fwd_qkvpacked(
+        qkv.data_ptr(), out.data_ptr(), None if lse is None else lse.data_ptr(), B, N, H, d,
+        0.0 if softmax_scale is None else float(softmax_scale), int(bool(causal)),
+        float(dropout_p), _DT[qkv.dtype], _stream_ptr(qkv))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_qkvpacked")
+    return out, lse
+
+
+def device_status(clear: bool = True):
+    """(status, detail) of the current device's watchdog word; synchronises."""
+    detail = ctypes.c_uint(0)
+    rc = load().fa_device_status(int(bool(clear)), ctypes.byref(detail))
+    return int(rc), int(detail.value)
+
+
+def watchdog_selftest(limit_ns: int = 20_000_000):
+    """Run the bounded-wait self test kernel on the current stream."""
+    rc = load().fa_debug_watchdog_selftest(int(limit_ns),
+                                           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_debug_watchdog_selftest")
+
+
+def launch_ctas(B: int, H: int, N: int, d: int, causal: bool = False) -> int:
+    return int(load().fa_launch_ctas(B, H, N, d, int(bool(causal))))
+
+
+def default_scale(d: int) -> float:
+    """The fp32 scale the library uses when none is given: 1/sqrt(d) rounded to fp32."""
+    return float(torch.tensor(1.0 / math.sqrt(d), dtype=torch.float32))

@@ -1,0 +1,121 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention forward library
+ * (libfa_sm100.so).
+ *
+ * Operation.  For every batch b, head h and query row i:
+ *
+ *     s_j    = scale * sum_c q[b,h,i,c] * k[b,h,j,c]      (key j visible from i)
+ *     O[i]   = sum_j exp(s_j) v[b,h,j,:] / sum_j exp(s_j)
+ *     LSE[i] = ln sum_j exp(s_j)
+ *
+ * i.e. O = softmax(scale * Q K^T [+ causal mask]) V, the standard attention of
+ * "2.3 FlashAttention与IO感知注意力(1)" (aiknowledge.cn), section 1.1, and of
+ * standard_attention in "flash_attention.py" (forceinjection.github.io),
+ * computed with the tiled online-softmax recurrence of flash_attention_forward
+ * in the same file, so the N x N score matrix never reaches device memory.
+ * With causal != 0, key j is visible from query i iff j <= i (lower triangle
+ * including the diagonal).  LSE is the natural-log logsumexp of the scaled
+ * scores over the visible keys, stored in fp32.
+ *
+ * Precision.  Inputs and O are fp16 or bf16; scores, the softmax state and the
+ * O accumulator are fp32; the softmax weights P are rounded to the input type
+ * before the P V product (as on the tensor cores of every FlashAttention).
+ *
+ * Memory.  Every pointer is device memory owned by the caller; the library
+ * allocates nothing per call.  q, k, v, qkv and o must be 16-byte aligned.
+ *
+ * Execution.  Calls are asynchronous on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream) and never synchronise.  The returned status covers
+ * argument checks and the launch only; a kernel whose bounded internal wait
+ * ran out (which does not happen in correct operation) is reported by
+ * fa_device_status().
+ *
+ * Errors are returned, never raised: no call aborts the process.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+
+enum fa_status {
+  FA_OK = 0,
+  FA_ERR_ARG = -1,         /* null pointer, B/H/N < 1, bad scale, size overflow */
+  FA_ERR_ALIGN = -2,       /* a tensor pointer is not 16-byte aligned */
+  FA_ERR_HEADDIM = -3,     /* d is not 64, 128 or 256 */
+  FA_ERR_DTYPE = -4,       /* dtype is not FA_FP16 or FA_BF16 */
+  FA_ERR_UNSUPPORTED = -5, /* dropout_p != 0 */
+  FA_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
+  FA_ERR_TIMEOUT = -7,     /* a kernel gave up on a bounded wait */
+  FA_ERR_DEVICE = -8       /* the current device is not sm_100 (B200 class) */
+};
+
+enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1 };
+
+/*
+ * Attention forward on separate Q, K, V.
+ *
+ *   q, k, v : [B, H, N, d] contiguous, element type `dtype` (read only)
+ *   o       : [B, H, N, d] contiguous, element type `dtype` (written)
+ *   lse     : [B, H, N] fp32 (written), or NULL to skip it
+ *   d       : 64, 128 or 256 (the head dims up to 256 that the feature list of
+ *             "flash-attention与TensorRT 10集成", blog.gitcode.com, names)
+ *   scale   : logit scale; 0 means 1/sqrt(d) (softmax_scale=None of the packed
+ *             call in section 5.2 of the intelliparadigm.com build guide).
+ *             Negative, NaN and infinite values are rejected.
+ *   causal  : 0 or 1
+ *
+ * Signature as the flash_attn_func(q, k, v) call of section 11.1 of the
+ * intelliparadigm.com guide, in the [B, H, N, d] layout of the aiknowledge.cn
+ * page, section 1.1.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H, int N,
+           int d, float scale, int causal, int dtype, struct CUstream_st *stream);
+
+/*
+ * Attention forward on a packed QKV tensor, as flash_attn_qkvpacked_func in
+ * section 5.2 (and the keyword list of section 10.1) of
+ * "Windows下RTX 3090编译Flash Attention 2.8.3全指南" (intelliparadigm.com).
+ *
+ *   qkv       : [B, N, 3, H, d] contiguous; index 0 / 1 / 2 of axis 2 is q / k / v
+ *   o         : [B, N, H, d] contiguous (written)
+ *   lse       : [B, H, N] fp32 (written), or NULL
+ *   dropout_p : must be 0 (dropout is not part of this forward); else FA_ERR_UNSUPPORTED
+ *   other arguments as fa_fwd.
+ */
+int fa_fwd_qkvpacked(const void *qkv, void *o, float *lse, int B, int N, int H, int d, float scale,
+                     int causal, float dropout_p, int dtype, struct CUstream_st *stream);
+
+/* Static text for a status code. */
+const char *fa_strerror(int status);
+
+/*
+ * Reads (and, if clear != 0, resets) the current device's watchdog word.
+ * Synchronises the current device first.  Returns FA_OK, FA_ERR_TIMEOUT when a
+ * kernel gave up on a bounded wait (`*detail`, if not NULL, receives the
+ * (role << 8) | site code), or FA_ERR_CUDA.
+ */
+int fa_device_status(int clear, unsigned int *detail);
+
+/*
+ * Launches a one-warp kernel that waits on a barrier nobody arrives at, with a
+ * bound of `limit_ns` nanoseconds.  The wait gives up, records FA_ERR_TIMEOUT in
+ * the watchdog word and the kernel returns normally.  For testing the failure
+ * path without a hang.  Returns the launch status.
+ */
+int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st *stream);
+
+/* Grid size (CTAs) fa_fwd would launch for this problem on the current device, or < 0. */
+int fa_launch_ctas(int B, int H, int N, int d, int causal);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */

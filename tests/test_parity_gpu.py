@@ -1,0 +1,166 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small shapes are compared on every output element; they span several 128-row
+tiles, ragged tails and the degenerate sizes (N = 1, one key block, one query
+tile in a two-tile work unit).  Bounds: O max-abs <= 2e-2 and mean-abs <= 2e-3,
+LSE within 1e-3 relative (|dLSE| <= 1e-3 * max(1, |LSE|)).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_154_b200 import fa, synth
+from exact_attention_154_b200.synth import BF16, FP16
+
+from parity import check
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    fa.load()
+    yield
+    rc, detail = fa.device_status(clear=True)
+    assert rc == fa.FA_OK, f"watchdog fired: {detail:#x}"
+
+
+def run_fwd(q, k, v, causal, scale=None):
+    o, lse = fa.fwd(q.cuda(), k.cuda(), v.cuda(), scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    return o.cpu(), lse.cpu()
+
+
+SMALL_N = [1, 7, 64, 127, 128, 129, 200, 256, 257, 300, 513]
+
+
+@pytest.mark.parametrize("dtype", [FP16, BF16])
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", SMALL_N)
+def test_small_shapes_full(N, d, causal, dtype):
+    B, H = 2, 2
+    q, k, v = synth.random_inputs(B, H, N, d, dtype, seed=1000 + N + d + int(causal))
+    o, lse = run_fwd(q, k, v, causal)
+    check(o, lse, q, k, v, fa.default_scale(d), causal, label=f"N={N} d={d} causal={causal}")
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_explicit_scale_and_large_logits(d):
+    N = 384
+    q, k, v = synth.random_inputs(1, 2, N, d, BF16, seed=77, sigma_qk=3.0)
+    for scale in (0.05, 1.0 / math.sqrt(d)):
+        o, lse = run_fwd(q, k, v, False, scale=scale)
+        sc = float(torch.tensor(scale, dtype=torch.float32))
+        check(o, lse, q, k, v, sc, False, label=f"scale={scale}")
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_closed_forms_on_gpu(causal):
+    d, N = 128, 300
+    g = torch.Generator().manual_seed(5)
+    # all keys equal -> O is the mean of the visible V rows
+    q = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 1, 1, d, generator=g).to(torch.bfloat16).expand(1, 1, N, d).contiguous()
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    o, lse = run_fwd(q, k, v, causal)
+    vd = v.double()[0, 0]
+    counts = torch.arange(1, N + 1, dtype=torch.float64)[:, None]
+    mean = (vd.cumsum(0) / counts) if causal else vd.mean(0, keepdim=True).expand(N, d)
+    assert (o.double()[0, 0] - mean).abs().max() < 2e-2
+    # causal row 0 sees only key 0 -> O[0] == V[0] exactly (after rounding)
+    if causal:
+        q2, k2, v2 = synth.random_inputs(1, 3, N, d, BF16, seed=9, sigma_qk=3.0)
+        o2, _ = run_fwd(q2, k2, v2, True)
+        assert torch.equal(o2[:, :, 0], v2[:, :, 0])
+
+
+def test_n1_returns_v():
+    for d in (64, 128, 256):
+        q, k, v = synth.random_inputs(3, 2, 1, d, FP16, seed=3)
+        o, lse = run_fwd(q, k, v, False)
+        assert torch.equal(o, v)
+        ref = (q.double() * k.double()).sum(-1) * fa.default_scale(d)
+        assert (lse.double() - ref).abs().max() < 1e-3
+
+
+def test_constant_v():
+    q, k, _ = synth.random_inputs(1, 2, 777, 128, BF16, seed=11)
+    v = torch.full_like(q, 0.75)
+    o, _ = run_fwd(q, k, v, True)
+    assert (o.double() - 0.75).abs().max() < 4e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_packed_layout(causal):
+    w = synth.packed_qkv_b2_n256_h12()
+    (qkv,) = synth.make_inputs(w)
+    o, lse = fa.fwd_qkvpacked(qkv.cuda(), dropout_p=0.0, softmax_scale=None, causal=causal)
+    torch.cuda.synchronize()
+    q, k, v = synth.unpack_qkv(qkv)
+    check(o.cpu().permute(0, 2, 1, 3), lse.cpu(), q, k, v, fa.default_scale(w.d), causal,
+          label="packed")
+
+
+def test_packed_ragged_and_d128():
+    g = torch.Generator().manual_seed(21)
+    qkv = torch.randn(3, 333, 3, 5, 128, generator=g).to(torch.bfloat16)
+    o, lse = fa.fwd_qkvpacked(qkv.cuda(), causal=True)
+    torch.cuda.synchronize()
+    q, k, v = synth.unpack_qkv(qkv)
+    check(o.cpu().permute(0, 2, 1, 3), lse.cpu(), q, k, v, fa.default_scale(128), True,
+          label="packed ragged")
+
+
+def test_no_lse_and_preallocated_out():
+    q, k, v = synth.random_inputs(1, 2, 300, 64, FP16, seed=31)
+    qc, kc, vc = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty_like(qc)
+    o, lse = fa.fwd(qc, kc, vc, causal=True, out=out, return_lse=False)
+    assert lse is None and o.data_ptr() == out.data_ptr()
+    o2, _ = fa.fwd(qc, kc, vc, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2)
+
+
+def test_deterministic():
+    q, k, v = (t.cuda() for t in synth.random_inputs(2, 4, 1000, 128, BF16, seed=41))
+    o1, l1 = fa.fwd(q, k, v, causal=True)
+    o2, l2 = fa.fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_many_tiles_more_than_sms():
+    # more work tiles than SMs: every CTA walks several tiles
+    q, k, v = synth.random_inputs(2, 80, 520, 128, BF16, seed=51)
+    o, lse = run_fwd(q, k, v, True)
+    rows = [0, 1, 127, 128, 255, 256, 300, 511, 519]
+    check(o, lse, q, k, v, fa.default_scale(128), True, rows=rows, label="many tiles")
+
+
+def test_stream_semantics():
+    q, k, v = (t.cuda() for t in synth.random_inputs(1, 4, 640, 64, BF16, seed=61))
+    s = torch.cuda.Stream()
+    ref, _ = fa.fwd(q, k, v)
+    with torch.cuda.stream(s):
+        o, _ = fa.fwd(q, k, v)
+    s.synchronize()
+    assert torch.equal(o, ref)
+
+
+def test_watchdog_gives_up_and_reports():
+    rc, _ = fa.device_status(clear=True)
+    assert rc == fa.FA_OK
+    fa.watchdog_selftest(limit_ns=20_000_000)
+    rc, detail = fa.device_status(clear=True)
+    assert rc == fa.FA_ERR_TIMEOUT and detail == (4 << 8) | 8
+    # the context is still usable afterwards
+    q, k, v = synth.random_inputs(1, 1, 200, 64, FP16, seed=71)
+    o, lse = run_fwd(q, k, v, False)
+    check(o, lse, q, k, v, fa.default_scale(64), False, label="after watchdog")
+    assert fa.device_status(clear=True)[0] == fa.FA_OK
