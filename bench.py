@@ -34,6 +34,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from exact_attention_154_b200 import dist as fdist  # noqa: E402
 from exact_attention_154_b200 import fa, synth  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense tensor-core peak"
@@ -165,18 +166,11 @@ def dist_setup():
 
 
 def dist_max(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return fdist.max_over_ranks(x, world, device="cuda")
 
 
 def dist_barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    fdist.barrier(world)
 
 
 def device_inputs(w):
@@ -316,6 +310,7 @@ def clocks_ok(c):
 
 
 def bench_gpu(args, w, key, world, rank, local):
+    w = fdist.shard_workload(w, world, rank)
     dev_in = device_inputs(w)
     go, _ = launcher(w, dev_in)
     flops = w.flops
