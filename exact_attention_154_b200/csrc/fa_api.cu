@@ -248,6 +248,15 @@ int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st* 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_debug_exp2_poly(const float* x, float* y, int n, struct CUstream_st* stream) {
+  if (!x || !y || n < 0) return FA_ERR_ARG;
+  if (n == 0) return FA_OK;
+  const int threads = 256, pairs = (n + 1) / 2;
+  exp2_poly_kernel<<<(pairs + threads - 1) / threads, threads, 0,
+                     reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_launch_ctas(int B, int H, int N, int d, int causal) {
   float scale = 0.f;
   int rc = check_common(B, H, N, d, &scale, causal, FA_BF16);

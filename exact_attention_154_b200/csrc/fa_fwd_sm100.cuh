@@ -43,6 +43,11 @@ namespace fa_sm100 {
 constexpr int BM = 128;  // query rows per Q tile (tcgen05 M)
 constexpr int BN = 128;  // key / value rows per K or V tile
 constexpr float kLazyRescaleLog2 = 8.0f;
+// Argument pairs (of every 8) whose exp2 runs on the FMA pipe instead of MUFU.
+#ifndef FA_POLY_PAIRS_PER8
+#define FA_POLY_PAIRS_PER8 2
+#endif
+constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;
 
 // Error word written by a kernel whose bounded wait ran out: 0 = none,
 // otherwise (role << 8) | site, first writer wins.
@@ -98,14 +103,16 @@ struct FwdCfg {
   static constexpr int SOFTMAX_WARPS = 4 * QS;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
-  static constexpr int THREADS = 32 * (SOFTMAX_WARPS + 2);
+  // whole warpgroups: the softmax groups, then one group holding the producer
+  // warp, the MMA warp and two idle warps
+  static constexpr int THREADS = 128 * (QS + 1);
 
   static constexpr int SQ_OFF = 0;
   static constexpr int SKV_OFF = QS * TILE_BYTES;
   static constexpr int BAR_OFF = SKV_OFF + KVS * TILE_BYTES;
   // barrier indices
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_KV_FULL = 2, B_KV_EMPTY = 2 + KVS,
-                       B_S_FULL = 2 + 2 * KVS, B_P_FULL = B_S_FULL + 2, B_O_DONE = B_P_FULL + 2,
+                       B_S_FULL = 2 + 2 * KVS, B_P_FULL = B_S_FULL + 2, B_O_DONE = B_P_FULL + 4,
                        B_DRAIN = B_O_DONE + 2, NUM_BARS = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-B alignment
@@ -217,8 +224,9 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
   if (!ok) {
     // Let the loads already issued land before the CTA's shared memory goes away.
     const unsigned long long drain = 10000000ull;
+    volatile int no_abort_q = 0;
     if (q_count > 0)
-      wait_phase(bars + 8 * C::B_Q_FULL, (q_count - 1) & 1, abort_flag, drain,
+      wait_phase(bars + 8 * C::B_Q_FULL, (q_count - 1) & 1, &no_abort_q, drain,
                  (kRoleProducer << 8) | kSiteDrain);
     for (int i = max(0, kv_count - KVS); i < kv_count; ++i) {
       volatile int no_abort = 0;
@@ -259,12 +267,26 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
              idesc_qk, kk > 0 ? 1u : 0u);
     }
   };
-  auto issue_pv = [&](uint32_t o_col, uint32_t p_col, int vslot, bool accumulate) {
+  // O (+)= P V, P handed over in two halves of 64 keys: the first four K-steps
+  // start as soon as the softmax has written the first half.
+  auto issue_pv = [&](int bar, uint32_t o_col, uint32_t p_col, int vslot, bool accumulate) -> bool {
     const uint32_t vb = base + C::SKV_OFF + vslot * C::TILE_BYTES;
 #pragma unroll
-    for (int kk = 0; kk < BN / 16; ++kk)
-      mma_ts(tmem + o_col, tmem + p_col + kk * 8, sw128_desc(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024),
-             idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+    for (int half = 0; half < 2; ++half) {
+      if (!wait_phase(bars + 8 * (C::B_P_FULL + 2 * bar + half), p_par[bar], abort_flag, lim,
+                      (kRoleMma << 8) | kSitePFull))
+        return false;
+      tc_fence_after_sync();
+#pragma unroll
+      for (int k4 = 0; k4 < BN / 32; ++k4) {
+        const int kk = half * (BN / 32) + k4;
+        mma_ts(tmem + o_col, tmem + p_col + kk * 8,
+               sw128_desc(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024), idesc_pv,
+               (accumulate || kk > 0) ? 1u : 0u);
+      }
+    }
+    p_par[bar] ^= 1u;
+    return true;
   };
 
   for (int round = 0; ok && round * G < p.num_tiles; ++round) {
@@ -280,21 +302,21 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     for (int j = 0; ok && j <= ti.n_max; ++j) {
       const int k_idx = kv0 + 2 * j, v_idx = kv0 + 2 * j - 1;
       if constexpr (QS == 2) {
+        // order: PV0(j-1), S0(j), PV1(j-1), S1(j)
         if (j >= 1 && !(ok = wait_kv(v_idx))) break;
-        if (j < ti.n_max && !(ok = wait_kv(k_idx))) break;
+        bool k_ready = false;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
           const uint32_t o_col = s ? C::O_COL1 : C::O_COL0;
           if (j >= 1 && j <= ti.n[s]) {
-            ok = wait_phase(bars + 8 * (C::B_P_FULL + s), p_par[s], abort_flag, lim,
-                            (kRoleMma << 8) | kSitePFull);
-            p_par[s] ^= 1u;
-            tc_fence_after_sync();
-            if (!ok) break;
-            issue_pv(o_col, C::s_col(s), v_idx % KVS, j > 1);
+            if (!(ok = issue_pv(s, o_col, C::s_col(s), v_idx % KVS, j > 1))) break;
             tc_commit(bars + 8 * (C::B_O_DONE + s));
           }
           if (j < ti.n[s]) {
+            if (!k_ready) {
+              if (!(ok = wait_kv(k_idx))) break;
+              k_ready = true;
+            }
             issue_s(s, C::s_col(s), k_idx % KVS);
             tc_commit(bars + 8 * (C::B_S_FULL + s));
           }
@@ -304,6 +326,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         if (j >= 1) tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
         if (j == ti.n_max - 1) tc_commit(bars + 8 * C::B_Q_EMPTY);
       } else {
+        // order: S(j) into the other S buffer, then PV(j-1)
         if (j < ti.n_max) {
           if (!(ok = wait_kv(k_idx))) break;
           const int buf = s_iter & 1;
@@ -315,12 +338,7 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         }
         if (j >= 1) {
           if (!(ok = wait_kv(v_idx))) break;
-          ok = wait_phase(bars + 8 * C::B_P_FULL, p_par[0], abort_flag, lim,
-                          (kRoleMma << 8) | kSitePFull);
-          p_par[0] ^= 1u;
-          tc_fence_after_sync();
-          if (!ok) break;
-          issue_pv(C::O_COL0, C::s_col(pv_iter & 1), v_idx % KVS, j > 1);
+          if (!(ok = issue_pv(0, C::O_COL0, C::s_col(pv_iter & 1), v_idx % KVS, j > 1))) break;
           tc_commit(bars + 8 * C::B_O_DONE);
           tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
           ++pv_iter;
@@ -334,6 +352,57 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     volatile int no_abort = 0;
     tc_commit(bars + 8 * C::B_DRAIN);
     wait_phase(bars + 8 * C::B_DRAIN, 0, &no_abort, 10000000ull, (kRoleMma << 8) | kSiteDrain);
+  }
+}
+
+// 2^x for two arguments on the FMA pipe: x = n + f with n = rint(x) taken from
+// the low mantissa bits of x + 1.5 * 2^23, f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial whose coefficients are the relative-error minimax fit on
+// [-1/2, 1/2] (Remez exchange, max relative error 7.5e-5, below half an ulp of
+// bf16 and fp16 P); 2^n applied by adding n to the exponent field.  Arguments
+// are clamped at -126 so the exponent cannot wrap (2^-126 is ~0 here).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f,
+                  c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+  float2 q = __ffma2_rn(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = __ffma2_rn(q, f, make_float2(c1, c1));
+  q = __ffma2_rn(q, f, make_float2(c0, c0));
+  float2 r;
+  r.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+  r.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+  return r;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Exponentials, row-sum and 16-bit packing of 32 consecutive scores.
+// POLY8 of every 8 argument pairs go through exp2_poly2, the rest through ex2.
+template <bool BF16, int POLY8>
+__device__ __forceinline__ void softmax_chunk(const float* sv, float sl2, float neg_ref,
+                                              uint32_t* pk, float2& acc) {
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const float2 x = __ffma2_rn(make_float2(sv[2 * q], sv[2 * q + 1]), make_float2(sl2, sl2),
+                               make_float2(neg_ref, neg_ref));
+    float2 e;
+    if ((q % 8) >= 8 - POLY8) {
+      e = exp2_poly2(x);
+    } else {
+      e.x = ex2(x.x);
+      e.y = ex2(x.y);
+    }
+    acc = __fadd2_rn(acc, e);
+    pk[q] = pack2<BF16>(e.x, e.y);
   }
 }
 
@@ -387,15 +456,17 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
 #pragma unroll
         for (int c = 0; c < 128; ++c) sv[c] = (c < lim_local) ? sv[c] : -INFINITY;
       }
-      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+      float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, sv[c]);
-        mx1 = fmaxf(mx1, sv[c + 1]);
-        mx2 = fmaxf(mx2, sv[c + 2]);
-        mx3 = fmaxf(mx3, sv[c + 3]);
+      for (int c = 4; c < 124; c += 8) {
+        mx[0] = max3(mx[0], sv[c], sv[c + 4]);
+        mx[1] = max3(mx[1], sv[c + 1], sv[c + 5]);
+        mx[2] = max3(mx[2], sv[c + 2], sv[c + 6]);
+        mx[3] = max3(mx[3], sv[c + 3], sv[c + 7]);
       }
-      const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_blk =
+          max3(max3(mx[0], mx[1], sv[124]), max3(mx[2], mx[3], sv[125]), fmaxf(sv[126], sv[127])) *
+          sl2;
 
       float alpha = 1.f;
       bool rescale = false;
@@ -408,21 +479,6 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       }
       const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
 
-      float sum0 = 0.f, sum1 = 0.f;
-      uint32_t pk[64];
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(fmaf(sv[c], sl2, neg_ref));
-        const float p1 = ex2(fmaf(sv[c + 1], sl2, neg_ref));
-        sum0 += p0;
-        sum1 += p1;
-        pk[c / 2] = pack2<BF16>(p0, p1);
-      }
-      l = l * alpha + (sum0 + sum1);
-      // P (128 x 16-bit per row = 64 columns) goes over the start of the S buffer.
-      tmem_st32(lane_base + s_col, pk);
-      tmem_st32(lane_base + s_col + 32, pk + 32);
-
       if (j > 0) {
         // O must hold every earlier P V product before it is rescaled.
         ok = wait_phase(bars + 8 * (C::B_O_DONE + bar_idx), o_par, abort_flag, lim,
@@ -432,19 +488,37 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         tc_fence_after_sync();
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
-          for (int c = 0; c < HD; c += 32) {
-            uint32_t ov[32];
-            tmem_ld32_sync(lane_base + o_col + c, ov);
+          for (int c = 0; c < HD; c += 16) {
+            uint32_t ov[16];
+            tmem_ld16_sync(lane_base + o_col + c, ov);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32(lane_base + o_col + c, ov);
+            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st16(lane_base + o_col + c, ov);
           }
         }
       }
-      tmem_st_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + bar_idx));
+
+      // P (128 x 16-bit per row = 64 columns) goes over the start of the S
+      // buffer, handed to the MMA warp in two halves of 64 keys.
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col = half * 64 + c * 32;
+          uint32_t pk[16];
+          if (need_mask)
+            softmax_chunk<BF16, 0>(sv + col, sl2, neg_ref, pk, acc);
+          else
+            softmax_chunk<BF16, kPolyPairsPer8>(sv + col, sl2, neg_ref, pk, acc);
+          tmem_st16(lane_base + s_col + col / 2, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + 2 * bar_idx + half));
+      }
+      l = l * alpha + (acc.x + acc.y);
       ++s_iter;
     }
 
@@ -503,9 +577,10 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars + 8 * (C::B_S_FULL + i), 1);
-      mbar_init(bars + 8 * (C::B_P_FULL + i), 4);  // one arrival per softmax warp
       mbar_init(bars + 8 * (C::B_O_DONE + i), 1);
     }
+    for (int i = 0; i < 4; ++i)  // [Q tile][half of P]: one arrival per softmax warp
+      mbar_init(bars + 8 * (C::B_P_FULL + i), 4);
     mbar_init(bars + 8 * C::B_DRAIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -528,9 +603,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
     softmax_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
   } else if (warp == C::PRODUCER_WARP) {
     if (lane == 0) producer_role<HD, QS, KVS, BF16>(p, base, abort_flag);
-  } else {
+  } else if (warp == C::MMA_WARP) {
     if (lane == 0) mma_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
-  }
+  }  // the remaining warps of the last warpgroup have no role
 
   tc_fence_before_sync();
   __syncthreads();
@@ -556,6 +631,18 @@ __global__ void watchdog_selftest_kernel(unsigned long long limit_ns) {
   if (threadIdx.x == 0)
     wait_phase(smem_u32(&bar), 0, &abort_word, limit_ns, (kRoleTest << 8) | kSiteSelfTest);
   __syncthreads();
+}
+
+// Evaluates exp2_poly2 on n arguments (test hook for the software exp2).
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
 }
 
 }  // namespace fa_sm100

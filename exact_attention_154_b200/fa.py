@@ -33,6 +33,7 @@ SIGNATURES = {
     "fa_device_status": (_I, [_I, ctypes.POINTER(ctypes.c_uint)]),
     "fa_debug_watchdog_selftest": (_I, [ctypes.c_ulonglong, _VP]),
     "fa_launch_ctas": (_I, [_I, _I, _I, _I, _I]),
+    "fa_debug_exp2_poly": (_I, [_VP, _VP, _I, _VP]),
     "fa_version": (_I, []),
 }
 
@@ -166,6 +167,17 @@ def watchdog_selftest(limit_ns: int = 20_000_000):
                                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_debug_watchdog_selftest")
+
+
+def exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """The kernel's software exp2 applied to a float32 CUDA tensor (test hook)."""
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    rc = load().fa_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(x))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_debug_exp2_poly")
+    return y
 
 
 def launch_ctas(B: int, H: int, N: int, d: int, causal: bool = False) -> int:

@@ -108,6 +108,13 @@ int fa_device_status(int clear, unsigned int *detail);
  */
 int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st *stream);
 
+/*
+ * Test hook: y[i] = the kernel's software 2^x (the FMA-pipe exponential used
+ * for part of the softmax weights) for n device floats x.  Not part of the
+ * attention method; exposed so that its error against exp2f can be measured.
+ */
+int fa_debug_exp2_poly(const float *x, float *y, int n, struct CUstream_st *stream);
+
 /* Grid size (CTAs) fa_fwd would launch for this problem on the current device, or < 0. */
 int fa_launch_ctas(int B, int H, int N, int d, int causal);
 

@@ -104,3 +104,8 @@ def test_library_has_no_torch_dependency():
     import subprocess
     out = subprocess.run(["ldd", fa.lib_path()], capture_output=True, text=True).stdout
     assert "torch" not in out and "python" not in out
+
+
+def test_exp2_hook_argument_check(lib):
+    assert lib.fa_debug_exp2_poly(None, P, 4, None) == fa.FA_ERR_ARG
+    assert lib.fa_debug_exp2_poly(P, P, -1, None) == fa.FA_ERR_ARG
