@@ -75,12 +75,12 @@ int device_state(DeviceState** out, int* dev_out) {
 }
 
 // 4-D view (d, N, H, B) of one operand with element strides (1, sn, sh, sb);
-// box of 64 elements (128 bytes) x 128 rows, 128-byte swizzle, zero fill.
+// box of 64 elements (128 bytes) x `rows` rows, 128-byte swizzle, zero fill.
 int encode_operand(CUtensorMap* map, const void* ptr, int dtype, int d, int N, int H, int B,
-                   long long sn, long long sh, long long sb) {
+                   long long sn, long long sh, long long sb, int rows) {
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)sn * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
-  const cuuint32_t box[4] = {64, 128, 1, 1};
+  const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUtensorMapDataType t =
       dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -93,7 +93,7 @@ int encode_operand(CUtensorMap* map, const void* ptr, int dtype, int d, int N, i
 // Kernel configuration per head dim: (Q tiles per work tile, K/V ring stages).
 template <int HD> struct Pick;
 template <> struct Pick<64> { static constexpr int QS = 2, KVS = 8; };
-template <> struct Pick<128> { static constexpr int QS = 2, KVS = 4; };
+template <> struct Pick<128> { static constexpr int QS = 2, KVS = 3; };
 template <> struct Pick<256> { static constexpr int QS = 1, KVS = 2; };
 
 int q_tiles_for(int d) { return d == 256 ? 1 : 2; }
@@ -147,9 +147,9 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
 
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((rc = encode_operand(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
   p.o = o;
   p.lse = lse;
   p.o_stride_n = osn;

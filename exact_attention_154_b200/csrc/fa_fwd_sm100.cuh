@@ -12,16 +12,23 @@
 //     (b, h, 256 query rows = two 128-row Q tiles, or one for head dim 256);
 //   * a TMA producer warp loads the Q tiles once per work tile and streams
 //     128-row K and V tiles through a ring of shared-memory stages guarded by
-//     full / empty mbarriers (128-byte swizzle, no cluster multicast);
-//   * one thread of the MMA warp issues tcgen05 MMAs: S = Q K^T from shared
-//     memory into tensor memory (TMEM), and O += P V with P read from TMEM and
-//     V from shared memory, committing each group to an mbarrier;
+//     full / empty mbarriers (128-byte swizzle, no cluster multicast), K one
+//     block ahead of V;
+//   * one thread of the MMA warp issues tcgen05 MMAs: S = Q K^T into tensor
+//     memory (TMEM) and O += P V, both from shared-memory operands, committing
+//     each group to an mbarrier;
 //   * each softmax warpgroup owns one Q tile: thread t of the group owns query
 //     row t (TMEM lane t), so row max and row sum need no shuffles.  It reads
-//     S from TMEM, applies scale (in the log2 domain), the causal / ragged
-//     mask, the online update, writes P as 16-bit pairs back over S in TMEM,
-//     rescales O in TMEM when its reference max moved, and finally writes
-//     O / l and the logsumexp.
+//     S from TMEM and at once releases the S buffer, so the tensor core can
+//     already compute the next block's S; then it applies scale (in the log2
+//     domain), the causal / ragged mask and the online update, writes P as
+//     16-bit values into shared memory in the layout the MMA reads, rescales O
+//     in TMEM when its reference max moved, and finally writes O / l and the
+//     logsumexp.
+//
+// Because S(j+1) is computed while the softmax of block j runs, the softmax
+// groups work back to back and the two of them overlap on every SM
+// sub-partition, which one warp alone cannot do for the exponential unit.
 //
 // The running max used as the exp2 reference is only moved when the block max
 // exceeds it by more than 2^8 (in log2 units 8): O, l and the reference stay
@@ -55,12 +62,12 @@ __device__ unsigned int g_fa_watchdog = 0u;
 
 enum WaitSite : unsigned {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteODone,
-  kSiteSelfTest, kSiteDrain
+  kSiteSelfTest, kSiteDrain, kSiteSFree, kSitePFree
 };
 enum Role : unsigned { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4 };
 
 struct FwdParams {
-  CUtensorMap tmap_q;  // 4-D (d, N, H, B) views of q, k, v, box (64, 128, 1, 1)
+  CUtensorMap tmap_q;  // 4-D (d, N, H, B) views of q, k, v; box 64 elements x 128 rows
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   void* o;
@@ -100,35 +107,47 @@ struct FwdCfg {
   static constexpr int CHUNKS = HD / 64;          // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = 128 * 128;   // one chunk of a 128-row tile
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
+  static constexpr int P_TILE_BYTES = (BN / 64) * CHUNK_BYTES;  // 128 x 128 16-bit P
   static constexpr int SOFTMAX_WARPS = 4 * QS;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
   // whole warpgroups: the softmax groups, then one group holding the producer
-  // warp, the MMA warp and two idle warps
+  // warp, the MMA warp and two warps without a role
   static constexpr int THREADS = 128 * (QS + 1);
 
   static constexpr int SQ_OFF = 0;
-  static constexpr int SKV_OFF = QS * TILE_BYTES;
+  static constexpr int SP_OFF = QS * TILE_BYTES;
+  static constexpr int SKV_OFF = SP_OFF + QS * P_TILE_BYTES;
   static constexpr int BAR_OFF = SKV_OFF + KVS * TILE_BYTES;
-  // barrier indices
+  // barrier indices ([Q tile] unless noted)
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_KV_FULL = 2, B_KV_EMPTY = 2 + KVS,
-                       B_S_FULL = 2 + 2 * KVS, B_P_FULL = B_S_FULL + 2, B_O_DONE = B_P_FULL + 4,
-                       B_DRAIN = B_O_DONE + 2, NUM_BARS = B_DRAIN + 1;
+                       B_S_FULL = 2 + 2 * KVS, B_S_FREE = B_S_FULL + 2,
+                       B_P_FULL = B_S_FREE + 2,  // [Q tile][half of P]
+                       B_P_FREE = B_P_FULL + 4, B_O_FINAL = B_P_FREE + 2,
+                       B_DRAIN = B_O_FINAL + 2, NUM_BARS = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-B alignment
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-  // TMEM columns (fp32 words): two S buffers, then the O accumulators.
+  // TMEM columns (fp32 words): one S buffer per Q tile, then the O accumulators.
   static constexpr uint32_t TMEM_COLS = 512;
-  __host__ __device__ static constexpr uint32_t s_col(int buf) { return buf ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t s_col(int tile) { return tile ? 128u : 0u; }
   static constexpr uint32_t O_COL0 = 256u;
   static constexpr uint32_t O_COL1 = 256u + HD;
-  static_assert(256 + QS * HD <= 512, "TMEM budget");
+  static_assert(128 * QS <= 256 && 256 + QS * HD <= 512, "TMEM budget");
 };
 
 struct TileInfo {
-  int b, h, q0, diag0, n[2], n_max;
+  int b, h, q0, n[2], n_max;
 };
+
+// Key blocks a 128-row Q tile starting at row r0 needs: all of them, or with
+// the causal mask those up to and including its diagonal.
+__device__ __forceinline__ int key_blocks(const FwdParams& p, int r0) {
+  const int nkv = (p.N + BN - 1) / BN;
+  if (r0 >= p.N) return 0;
+  return p.causal ? min(nkv, r0 / BN + 1) : nkv;
+}
 
 template <int QS>
 __device__ __forceinline__ TileInfo decode_tile(const FwdParams& p, int t) {
@@ -140,18 +159,16 @@ __device__ __forceinline__ TileInfo decode_tile(const FwdParams& p, int t) {
   ti.b = bh / p.H;
   ti.h = bh - ti.b * p.H;
   ti.q0 = qblock * BM * QS;
-  ti.diag0 = ti.q0 / BN;
-  const int nkv = (p.N + BN - 1) / BN;
-  ti.n_max = 0;
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    int n = 0;
-    if (s < QS && ti.q0 + s * BM < p.N) n = p.causal ? min(nkv, ti.diag0 + s + 1) : nkv;
-    ti.n[s] = n;
-    ti.n_max = max(ti.n_max, n);
-  }
+  ti.n[0] = key_blocks(p, ti.q0);
+  ti.n[1] = QS == 2 ? key_blocks(p, ti.q0 + BM) : 0;
+  ti.n_max = max(ti.n[0], ti.n[1]);
   return ti;
 }
+
+// Ring positions (from the work tile's first) of K(j) and V(j) when a work
+// tile streams K(0), then K(j+1), V(j) for j = 0 .. n-2, then V(n-1).
+__host__ __device__ __forceinline__ int ring_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__host__ __device__ __forceinline__ int ring_v(int j, int n) { return j < n - 1 ? 2 * j + 2 : 2 * n - 1; }
 
 // Static persistent schedule: round r hands tiles [r*G, (r+1)*G) to the G
 // CTAs, reversing the order on odd rounds so causal work evens out.
@@ -184,6 +201,21 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0, q_count = 0;
   bool ok = true;
+  // one K or V tile into the next ring slot
+  auto load_kv = [&](const CUtensorMap* map, int row0, const TileInfo& ti) -> bool {
+    const int slot = kv_count % KVS, use = kv_count / KVS;
+    if (use > 0 && !wait_phase(bars + 8 * (C::B_KV_EMPTY + slot), (use - 1) & 1, abort_flag,
+                               p.wait_limit_ns, (kRoleProducer << 8) | kSiteKvEmpty))
+      return false;
+    const uint32_t full = bars + 8 * (C::B_KV_FULL + slot);
+    mbar_arrive_expect_tx(full, C::TILE_BYTES);
+#pragma unroll
+    for (int c = 0; c < C::CHUNKS; ++c)
+      tma_load_4d(base + C::SKV_OFF + slot * C::TILE_BYTES + c * C::CHUNK_BYTES, map, full,
+                  c * 64, row0, ti.h, ti.b);
+    ++kv_count;
+    return true;
+  };
   for (int round = 0; ok && round * G < p.num_tiles; ++round) {
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
@@ -201,24 +233,10 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
         tma_load_4d(base + C::SQ_OFF + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tmap_q,
                     bars + 8 * C::B_Q_FULL, c * 64, ti.q0 + s * BM, ti.h, ti.b);
     ++q_count;
+    ok = load_kv(&p.tmap_k, 0, ti);
     for (int j = 0; ok && j < ti.n_max; ++j) {
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        const int slot = kv_count % KVS, use = kv_count / KVS;
-        if (use > 0) {
-          ok = wait_phase(bars + 8 * (C::B_KV_EMPTY + slot), (use - 1) & 1, abort_flag,
-                          p.wait_limit_ns, (kRoleProducer << 8) | kSiteKvEmpty);
-          if (!ok) break;
-        }
-        const uint32_t full = bars + 8 * (C::B_KV_FULL + slot);
-        mbar_arrive_expect_tx(full, C::TILE_BYTES);
-        const CUtensorMap* map = kv ? &p.tmap_v : &p.tmap_k;
-#pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_4d(base + C::SKV_OFF + slot * C::TILE_BYTES + c * C::CHUNK_BYTES, map, full,
-                      c * 64, j * BN, ti.h, ti.b);
-        ++kv_count;
-      }
+      if (j + 1 < ti.n_max && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
+      ok = load_kv(&p.tmap_v, j * BN, ti);
     }
   }
   if (!ok) {
@@ -237,6 +255,10 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
   }
 }
 
+// Issue order per work tile (Q tile s = 0, 1; key block j):
+//   S_s(0)
+//   for each j:  S_s(j+1) once the softmax of tile s has read S_s(j),
+//                then P V_s(j) once it has written P_s(j).
 template <int HD, int QS, int KVS, bool BF16>
 __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
                          volatile int* abort_flag) {
@@ -247,8 +269,8 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const unsigned long long lim = p.wait_limit_ns;
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0, q_count = 0;
-  uint32_t p_par[2] = {0u, 0u};
-  int s_iter = 0, pv_iter = 0;  // single-Q-tile variant: S buffer ring position
+  uint32_t p_par[2] = {0u, 0u}, sf_par[2] = {0u, 0u};
+  int s_issued[2] = {0, 0};
   bool ok = true;
 
   auto wait_kv = [&](int idx) -> bool {
@@ -257,35 +279,51 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     tc_fence_after_sync();
     return r;
   };
-  auto issue_s = [&](int s, uint32_t s_col, int kslot) {
-    const uint32_t qa = base + C::SQ_OFF + s * C::TILE_BYTES;
-    const uint32_t kb = base + C::SKV_OFF + kslot * C::TILE_BYTES;
+  // S_s = Q_s K^T into the tile's S buffer, after the softmax has read the
+  // buffer's previous contents.  Descriptors are formed once per operand;
+  // the K-steps add constant offsets to the low word.
+  auto issue_s = [&](int s, int kslot) -> bool {
+    if (s_issued[s] > 0) {
+      if (!wait_phase(bars + 8 * (C::B_S_FREE + s), sf_par[s], abort_flag, lim,
+                      (kRoleMma << 8) | kSiteSFree))
+        return false;
+      sf_par[s] ^= 1u;
+      tc_fence_after_sync();
+    }
+    const uint32_t qa = sw128_desc_lo(base + C::SQ_OFF + s * C::TILE_BYTES, 16);
+    const uint32_t kb = sw128_desc_lo(base + C::SKV_OFF + kslot * C::TILE_BYTES, 16);
+    const uint32_t d_tmem = tmem + C::s_col(s);
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint32_t off = (kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32;
-      mma_ss(tmem + s_col, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + off, 16, 1024),
-             idesc_qk, kk > 0 ? 1u : 0u);
+      const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
+      mma_ss(d_tmem, desc_from_lo(qa + off), desc_from_lo(kb + off), idesc_qk, kk > 0 ? 1u : 0u);
     }
+    tc_commit(bars + 8 * (C::B_S_FULL + s));
+    ++s_issued[s];
+    return true;
   };
-  // O (+)= P V, P handed over in two halves of 64 keys: the first four K-steps
-  // start as soon as the softmax has written the first half.
-  auto issue_pv = [&](int bar, uint32_t o_col, uint32_t p_col, int vslot, bool accumulate) -> bool {
-    const uint32_t vb = base + C::SKV_OFF + vslot * C::TILE_BYTES;
+  // O (+)= P V with P read from shared memory, handed over in two halves of
+  // 64 keys: the first four K-steps start once the first half is written.
+  auto issue_pv = [&](int s, int vslot, bool accumulate) -> bool {
+    const uint32_t pa = sw128_desc_lo(base + C::SP_OFF + s * C::P_TILE_BYTES, 16);
+    const uint32_t vb = sw128_desc_lo(base + C::SKV_OFF + vslot * C::TILE_BYTES, C::CHUNK_BYTES);
+    const uint32_t d_tmem = tmem + (s ? C::O_COL1 : C::O_COL0);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      if (!wait_phase(bars + 8 * (C::B_P_FULL + 2 * bar + half), p_par[bar], abort_flag, lim,
+      if (!wait_phase(bars + 8 * (C::B_P_FULL + 2 * s + half), p_par[s], abort_flag, lim,
                       (kRoleMma << 8) | kSitePFull))
         return false;
       tc_fence_after_sync();
 #pragma unroll
-      for (int k4 = 0; k4 < BN / 32; ++k4) {
-        const int kk = half * (BN / 32) + k4;
-        mma_ts(tmem + o_col, tmem + p_col + kk * 8,
-               sw128_desc(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024), idesc_pv,
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = half * 4 + k4;
+        mma_ss(d_tmem, desc_from_lo(pa + ((half * C::CHUNK_BYTES + k4 * 32) >> 4)),
+               desc_from_lo(vb + ((kk * 16 * 128) >> 4)), idesc_pv,
                (accumulate || kk > 0) ? 1u : 0u);
       }
     }
-    p_par[bar] ^= 1u;
+    p_par[s] ^= 1u;
+    tc_commit(bars + 8 * (C::B_P_FREE + s));
     return true;
   };
 
@@ -298,54 +336,39 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     tc_fence_after_sync();
     ++q_count;
     if (!ok) break;
-    const int kv0 = kv_count;
-    for (int j = 0; ok && j <= ti.n_max; ++j) {
-      const int k_idx = kv0 + 2 * j, v_idx = kv0 + 2 * j - 1;
-      if constexpr (QS == 2) {
-        // order: PV0(j-1), S0(j), PV1(j-1), S1(j)
-        if (j >= 1 && !(ok = wait_kv(v_idx))) break;
-        bool k_ready = false;
+    const int kv0 = kv_count, n_max = ti.n_max;
+    // S(0)
+    if (!(ok = wait_kv(kv0 + ring_k(0)))) break;
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const uint32_t o_col = s ? C::O_COL1 : C::O_COL0;
-          if (j >= 1 && j <= ti.n[s]) {
-            if (!(ok = issue_pv(s, o_col, C::s_col(s), v_idx % KVS, j > 1))) break;
-            tc_commit(bars + 8 * (C::B_O_DONE + s));
-          }
-          if (j < ti.n[s]) {
-            if (!k_ready) {
-              if (!(ok = wait_kv(k_idx))) break;
-              k_ready = true;
-            }
-            issue_s(s, C::s_col(s), k_idx % KVS);
-            tc_commit(bars + 8 * (C::B_S_FULL + s));
-          }
-        }
+    for (int s = 0; s < QS; ++s)
+      if (ok && ti.n[s] > 0) ok = issue_s(s, (kv0 + ring_k(0)) % KVS);
+    if (!ok) break;
+    tc_commit(bars + 8 * (C::B_KV_EMPTY + (kv0 + ring_k(0)) % KVS));
+    if (n_max == 1) tc_commit(bars + 8 * C::B_Q_EMPTY);
+    for (int j = 0; ok && j < n_max; ++j) {
+      if (j + 1 < n_max) {  // S(j+1)
+        const int k_idx = kv0 + ring_k(j + 1);
+        if (!(ok = wait_kv(k_idx))) break;
+#pragma unroll
+        for (int s = 0; s < QS; ++s)
+          if (ok && j + 1 < ti.n[s]) ok = issue_s(s, k_idx % KVS);
         if (!ok) break;
-        if (j < ti.n_max) tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
-        if (j >= 1) tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
-        if (j == ti.n_max - 1) tc_commit(bars + 8 * C::B_Q_EMPTY);
-      } else {
-        // order: S(j) into the other S buffer, then PV(j-1)
-        if (j < ti.n_max) {
-          if (!(ok = wait_kv(k_idx))) break;
-          const int buf = s_iter & 1;
-          issue_s(0, C::s_col(buf), k_idx % KVS);
-          tc_commit(bars + 8 * (C::B_S_FULL + buf));
-          tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
-          if (j == ti.n_max - 1) tc_commit(bars + 8 * C::B_Q_EMPTY);
-          ++s_iter;
-        }
-        if (j >= 1) {
-          if (!(ok = wait_kv(v_idx))) break;
-          if (!(ok = issue_pv(0, C::O_COL0, C::s_col(pv_iter & 1), v_idx % KVS, j > 1))) break;
-          tc_commit(bars + 8 * C::B_O_DONE);
-          tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
-          ++pv_iter;
-        }
+        tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
+        if (j + 2 == n_max) tc_commit(bars + 8 * C::B_Q_EMPTY);
       }
+      // P V(j)
+      const int v_idx = kv0 + ring_v(j, n_max);
+      if (!(ok = wait_kv(v_idx))) break;
+#pragma unroll
+      for (int s = 0; s < QS; ++s)
+        if (ok && j < ti.n[s]) {
+          ok = issue_pv(s, v_idx % KVS, j > 0);
+          if (ok && j == ti.n[s] - 1) tc_commit(bars + 8 * (C::B_O_FINAL + s));
+        }
+      if (!ok) break;
+      tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
     }
-    kv_count = kv0 + 2 * ti.n_max;
+    kv_count = kv0 + 2 * n_max;
   }
   if (!ok) {
     // Wait for every MMA this thread issued before TMEM is released.
@@ -385,11 +408,40 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
+// Max of 128 scores as a balanced tree of 3-input maxima.
+__device__ __forceinline__ float row_max128(const float* sv) {
+  float t[43];
+#pragma unroll
+  for (int i = 0; i < 42; ++i) t[i] = max3(sv[3 * i], sv[3 * i + 1], sv[3 * i + 2]);
+  t[42] = fmaxf(sv[126], sv[127]);
+  float u[15];
+#pragma unroll
+  for (int i = 0; i < 14; ++i) u[i] = max3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+  u[14] = t[42];
+  float v[5];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) v[i] = max3(u[3 * i], u[3 * i + 1], u[3 * i + 2]);
+  return fmaxf(max3(v[0], v[1], v[2]), fmaxf(v[3], v[4]));
+}
+
+// Writes 64 keys of one P row (32 packed pairs) into the 128-byte swizzled,
+// K-major layout the P V MMA reads: row r of a 64-key chunk at r * 128 bytes,
+// its 16-byte group u at position u ^ (r % 8).
+__device__ __forceinline__ void store_p_chunk(uint32_t chunk_base, int r, const uint32_t* pk) {
+  const uint32_t row = chunk_base + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    st_shared_v4(row + ((static_cast<uint32_t>(u) ^ (r & 7u)) << 4), pk[4 * u], pk[4 * u + 1],
+                 pk[4 * u + 2], pk[4 * u + 3]);
+}
+
 // Exponentials, row-sum and 16-bit packing of 32 consecutive scores.
 // POLY8 of every 8 argument pairs go through exp2_poly2, the rest through ex2.
+// The row sum goes into four independent packed accumulators, so the adds
+// form four short dependency chains instead of one long one.
 template <bool BF16, int POLY8>
 __device__ __forceinline__ void softmax_chunk(const float* sv, float sl2, float neg_ref,
-                                              uint32_t* pk, float2& acc) {
+                                              uint32_t* pk, float2 (&acc)[4]) {
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     const float2 x = __ffma2_rn(make_float2(sv[2 * q], sv[2 * q + 1]), make_float2(sl2, sl2),
@@ -401,7 +453,7 @@ __device__ __forceinline__ void softmax_chunk(const float* sv, float sl2, float 
       e.x = ex2(x.x);
       e.y = ex2(x.y);
     }
-    acc = __fadd2_rn(acc, e);
+    acc[q & 3] = __fadd2_rn(acc[q & 3], e);
     pk[q] = pack2<BF16>(e.x, e.y);
   }
 }
@@ -416,13 +468,14 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const int s = warp / 4;                   // which Q tile of the work tile
   const int r = (warp % 4) * 32 + lane;     // query row within the tile == TMEM lane
   const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp % 4) * 32u) << 16);
+  const uint32_t s_col = C::s_col(s);
   const uint32_t o_col = s ? C::O_COL1 : C::O_COL0;
-  const int bar_idx = (QS == 2) ? s : 0;
+  const uint32_t sp = base + C::SP_OFF + s * C::P_TILE_BYTES;
   const unsigned long long lim = p.wait_limit_ns;
   const float sl2 = p.scale_log2;
   const int G = gridDim.x, cta = blockIdx.x;
-  uint32_t s_par[2] = {0u, 0u}, o_par = 0u;
-  int s_iter = 0;
+  uint32_t s_par = 0u, pf_par = 0u, fin_par = 0u;
+  int p_written = 0;  // P blocks this Q tile has handed to the MMA warp so far
 
   for (int round = 0; round * G < p.num_tiles; ++round) {
     const int t = tile_of(round, cta, G);
@@ -433,99 +486,92 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const int row = ti.q0 + s * BM + r;
     // keys visible from this row: [0, limit)
     const int limit = p.causal ? min(row + 1, p.N) : p.N;
+    // first key block that needs the mask
+    const int first_masked = p.causal ? ((ti.q0 + s * BM) / BN) : (p.N / BN);
     float m_ref = -INFINITY, l = 0.f;
 
     for (int j = 0; j < n; ++j) {
-      const int buf = (QS == 2) ? s : (s_iter & 1);
-      const uint32_t s_col = C::s_col(buf);
-      bool ok = wait_phase(bars + 8 * (C::B_S_FULL + buf), s_par[buf], abort_flag, lim,
+      bool ok = wait_phase(bars + 8 * (C::B_S_FULL + s), s_par, abort_flag, lim,
                            (kRoleSoftmax << 8) | kSiteSFull);
-      s_par[buf] ^= 1u;
+      s_par ^= 1u;
       if (!__all_sync(0xffffffffu, ok)) return;
       tc_fence_after_sync();
-
       uint32_t sr[128];
       tmem_ld128_sync(lane_base + s_col, sr);
+      // S is in registers: the MMA warp may overwrite the buffer with S(j+1).
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (C::B_S_FREE + s));
+
       float sv[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-
-      const bool need_mask = (p.causal && j >= ti.diag0 + s) || ((j + 1) * BN > p.N);
+      const bool need_mask = j >= first_masked;
       if (need_mask) {
         const int lim_local = limit - j * BN;
 #pragma unroll
         for (int c = 0; c < 128; ++c) sv[c] = (c < lim_local) ? sv[c] : -INFINITY;
       }
-      float mx[4] = {sv[0], sv[1], sv[2], sv[3]};
-#pragma unroll
-      for (int c = 4; c < 124; c += 8) {
-        mx[0] = max3(mx[0], sv[c], sv[c + 4]);
-        mx[1] = max3(mx[1], sv[c + 1], sv[c + 5]);
-        mx[2] = max3(mx[2], sv[c + 2], sv[c + 6]);
-        mx[3] = max3(mx[3], sv[c + 3], sv[c + 7]);
-      }
-      const float m_blk =
-          max3(max3(mx[0], mx[1], sv[124]), max3(mx[2], mx[3], sv[125]), fmaxf(sv[126], sv[127])) *
-          sl2;
+      const float m_blk = row_max128(sv) * sl2;
 
-      float alpha = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m_ref = m_blk;
-      } else if (m_blk > m_ref + kLazyRescaleLog2) {
-        alpha = ex2(m_ref - m_blk);
-        m_ref = m_blk;
-        rescale = true;
-      }
+      // Lazy reference: keep m_ref unless the block max exceeds it by more
+      // than 2^8; the first block always sets it.
+      const bool rescale = (j > 0) && (m_blk > m_ref + kLazyRescaleLog2);
+      const float m_new = (j == 0 || rescale) ? m_blk : m_ref;
+      const float alpha = (j == 0) ? 0.f : ex2(m_ref - m_new);  // 1 when m_ref is kept
+      m_ref = m_new;
       const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
 
-      if (j > 0) {
-        // O must hold every earlier P V product before it is rescaled.
-        ok = wait_phase(bars + 8 * (C::B_O_DONE + bar_idx), o_par, abort_flag, lim,
-                        (kRoleSoftmax << 8) | kSiteODone);
-        o_par ^= 1u;
-        if (!__all_sync(0xffffffffu, ok)) return;
-        tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-          for (int c = 0; c < HD; c += 16) {
-            uint32_t ov[16];
-            tmem_ld16_sync(lane_base + o_col + c, ov);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st16(lane_base + o_col + c, ov);
-          }
-        }
-      }
-
-      // P (128 x 16-bit per row = 64 columns) goes over the start of the S
-      // buffer, handed to the MMA warp in two halves of 64 keys.
-      float2 acc = make_float2(0.f, 0.f);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const int col = half * 64 + c * 32;
-          uint32_t pk[16];
           if (need_mask)
-            softmax_chunk<BF16, 0>(sv + col, sl2, neg_ref, pk, acc);
+            softmax_chunk<BF16, 0>(sv + 64 * half + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
           else
-            softmax_chunk<BF16, kPolyPairsPer8>(sv + col, sl2, neg_ref, pk, acc);
-          tmem_st16(lane_base + s_col + col / 2, pk);
+            softmax_chunk<BF16, kPolyPairsPer8>(sv + 64 * half + 32 * c, sl2, neg_ref,
+                                                pk + 16 * c, acc);
         }
-        tmem_st_wait();
+        if (half == 0) {
+          // The previous P V has finished: its P buffer is free and O holds it.
+          if (p_written > 0) {
+            ok = wait_phase(bars + 8 * (C::B_P_FREE + s), pf_par, abort_flag, lim,
+                            (kRoleSoftmax << 8) | kSitePFree);
+            pf_par ^= 1u;
+            if (!__all_sync(0xffffffffu, ok)) return;
+            tc_fence_after_sync();
+          }
+          if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+            for (int c = 0; c < HD; c += 16) {
+              uint32_t ov[16];
+              tmem_ld16_sync(lane_base + o_col + c, ov);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st16(lane_base + o_col + c, ov);
+            }
+            tmem_st_wait();
+          }
+        }
+        store_p_chunk(sp + half * C::CHUNK_BYTES, r, pk);
+        // make the generic-proxy stores visible to the tensor core
+        fence_proxy_async_smem();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + 2 * bar_idx + half));
+        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + 2 * s + half));
       }
-      l = l * alpha + (acc.x + acc.y);
-      ++s_iter;
+      ++p_written;
+      const float2 acc01 = __fadd2_rn(acc[0], acc[1]), acc23 = __fadd2_rn(acc[2], acc[3]);
+      l = l * alpha + ((acc01.x + acc23.x) + (acc01.y + acc23.y));
     }
 
     // Epilogue: wait for the last P V product, then O / l and the logsumexp.
-    bool ok = wait_phase(bars + 8 * (C::B_O_DONE + bar_idx), o_par, abort_flag, lim,
+    bool ok = wait_phase(bars + 8 * (C::B_O_FINAL + s), fin_par, abort_flag, lim,
                          (kRoleSoftmax << 8) | kSiteODone);
-    o_par ^= 1u;
+    fin_par ^= 1u;
     if (!__all_sync(0xffffffffu, ok)) return;
     tc_fence_after_sync();
     const float inv_l = 1.f / l;
@@ -550,7 +596,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       p.lse[(static_cast<long long>(ti.b) * p.H + ti.h) * p.N + row] =
           (m_ref + log2f(l)) * 0.69314718055994530942f;
     // The next tile's first P V overwrites O only after this group's next
-    // p_full arrival, which comes after these loads completed.
+    // P arrival, which comes after these loads completed.
     tc_fence_before_sync();
   }
 }
@@ -577,10 +623,11 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bars + 8 * (C::B_S_FULL + i), 1);
-      mbar_init(bars + 8 * (C::B_O_DONE + i), 1);
+      mbar_init(bars + 8 * (C::B_S_FREE + i), 4);  // one arrival per softmax warp
+      mbar_init(bars + 8 * (C::B_P_FREE + i), 1);
+      mbar_init(bars + 8 * (C::B_O_FINAL + i), 1);
     }
-    for (int i = 0; i < 4; ++i)  // [Q tile][half of P]: one arrival per softmax warp
-      mbar_init(bars + 8 * (C::B_P_FULL + i), 4);
+    for (int i = 0; i < 4; ++i) mbar_init(bars + 8 * (C::B_P_FULL + i), 4);
     mbar_init(bars + 8 * C::B_DRAIN, 1);
     *abort_flag = 0;
     fence_mbar_init();
