@@ -152,10 +152,20 @@ __device__ __forceinline__ int key_blocks(const FwdParams& p, int r0) {
 template <int QS>
 __device__ __forceinline__ TileInfo decode_tile(const FwdParams& p, int t) {
   TileInfo ti;
-  const int bh = t / p.num_qblocks;
-  const int qi = t - bh * p.num_qblocks;
-  // heaviest query blocks first within a head when causal
-  const int qblock = p.causal ? (p.num_qblocks - 1 - qi) : qi;
+  int bh, qblock;
+  if (p.causal) {
+    // longest first over the whole grid: all heads' last query block, then
+    // the one before, ...; with the snake hand-out below this balances the
+    // triangular work to within a few percent
+    const int nbh = p.B * p.H;
+    const int qi = t / nbh;
+    bh = t - qi * nbh;
+    qblock = p.num_qblocks - 1 - qi;
+  } else {
+    // equal work per tile: keep a head's query blocks together for K/V reuse in L2
+    bh = t / p.num_qblocks;
+    qblock = t - bh * p.num_qblocks;
+  }
   ti.b = bh / p.H;
   ti.h = bh - ti.b * p.H;
   ti.q0 = qblock * BM * QS;
@@ -171,7 +181,8 @@ __host__ __device__ __forceinline__ int ring_k(int j) { return j == 0 ? 0 : 2 * 
 __host__ __device__ __forceinline__ int ring_v(int j, int n) { return j < n - 1 ? 2 * j + 2 : 2 * n - 1; }
 
 // Static persistent schedule: round r hands tiles [r*G, (r+1)*G) to the G
-// CTAs, reversing the order on odd rounds so causal work evens out.
+// CTAs, reversing the order on odd rounds, so that with the longest-first
+// causal order every CTA gets a long and a short tile in each pair of rounds.
 __device__ __forceinline__ int tile_of(int round, int cta, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
