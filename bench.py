@@ -272,36 +272,44 @@ def row_flops(w, rows):
     return 4.0 * w.d * w.N * len(rows)
 
 
-def cpu_oracle_sample(w, target_s=12.0, max_rows_per_head=None):
-    """Times the fp64 oracle, as it stands, on a bounded sample of the
-    workload's query rows (the same rows in every (b, h)), on all host cores."""
-    import oracle
-    oracle.build()
-    if w.layout == "packed":
-        q, k, v = synth.unpack_qkv(synth.make_inputs(w)[0])
-    else:
-        q, k, v = synth.make_inputs(w)
-    q64, k64, v64 = (t.double().numpy() for t in (q, k, v))
-    rng = np.random.default_rng(w.seed + 2000)
-    sc = fa.default_scale(w.d)
+class OracleSampler:
+    """Times the fp64 oracle, as it stands, on bounded samples of the
+    workload's query rows (the same rows in every (b, h)), on all host cores.
+    The sample size is calibrated once so one timed call takes ~target_s."""
 
-    def run(nrows):
-        rows = np.sort(rng.choice(w.N, size=nrows, replace=False)).astype(np.int32)
+    def __init__(self, w, target_s):
+        import oracle
+        oracle.build()
+        self.oracle, self.w = oracle, w
+        if w.layout == "packed":
+            q, k, v = synth.unpack_qkv(synth.make_inputs(w)[0])
+        else:
+            q, k, v = synth.make_inputs(w)
+        self.qkv = tuple(t.double().numpy() for t in (q, k, v))
+        self.rng = np.random.default_rng(w.seed + 2000)
+        self.scale = fa.default_scale(w.d)
+        n0 = min(w.N, 2)
+        dt, _, _ = self.run(n0)
+        self.nrows = max(1, min(w.N, int(n0 * max(target_s, 1e-3) / max(dt, 1e-4))))
+
+    def run(self, nrows):
+        w = self.w
+        rows = np.sort(self.rng.choice(w.N, size=nrows, replace=False)).astype(np.int32)
         t0 = time.perf_counter()
-        oracle.attention(q64, k64, v64, scale=sc, causal=w.causal, rows=rows)
+        self.oracle.attention(*self.qkv, scale=self.scale, causal=w.causal, rows=rows)
         return time.perf_counter() - t0, row_flops(w, rows) * w.B * w.H, nrows
 
-    nrows = min(w.N, 4)
-    dt, fl, _ = run(nrows)
-    # grow the sample to about target_s seconds of CPU work
-    want = int(nrows * max(1.0, target_s / max(dt, 1e-3)))
-    cap = w.N if max_rows_per_head is None else min(w.N, max_rows_per_head)
-    nrows = max(1, min(cap, want))
-    dt, fl, nrows = run(nrows)
-    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle", "seconds": round(dt, 3),
-            "sample": f"{nrows} seeded query rows in each of the {w.B * w.H} (b, h) heads of "
-                      f"the workload (of N={w.N}), fp64 oracle, all host threads"}
+    def step(self):
+        dt, fl, nrows = self.run(self.nrows)
+        w = self.w
+        return {"value": fl / dt / 1e12, "unit": UNIT, "cores": self.oracle.num_threads(),
+                "kind": "oracle", "seconds": round(dt, 4),
+                "sample": f"{nrows} seeded query rows in each of the {w.B * w.H} (b, h) heads of "
+                          f"the workload (of N={w.N}), fp64 oracle, all host threads"}
+
+
+def cpu_oracle_sample(w, target_s=12.0):
+    return OracleSampler(w, target_s).step()
 
 
 def clocks_ok(c):
@@ -384,15 +392,13 @@ def main():
         if rank != 0:
             return 0
         w = table[args.workload]
-        per_step = []
-        info = None
-        for _ in range(args.warmup if args.warmup < 1 else 0):
-            pass
-        budget = max(2.0, 120.0 / max(1, args.steps + 1))
-        for _ in range(args.steps):
-            info = cpu_oracle_sample(w, target_s=min(budget, 10.0))
-            per_step.append(info["value"])
-        value = statistics.median(per_step)
+        # the whole --steps K --warmup W run stays within about two minutes
+        sampler = OracleSampler(w, target_s=min(10.0, 120.0 / max(1, args.steps + args.warmup)))
+        for _ in range(args.warmup):
+            sampler.step()
+        per_step = [sampler.step() for _ in range(args.steps)]
+        info = per_step[-1]
+        value = statistics.median(x["value"] for x in per_step)
         line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

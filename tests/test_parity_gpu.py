@@ -15,6 +15,7 @@ from exact_attention_154_b200 import fa, synth
 from exact_attention_154_b200.synth import BF16, FP16
 
 from parity import check
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -164,3 +165,24 @@ def test_watchdog_gives_up_and_reports():
     o, lse = run_fwd(q, k, v, False)
     check(o, lse, q, k, v, fa.default_scale(64), False, label="after watchdog")
     assert fa.device_status(clear=True)[0] == fa.FA_OK
+
+
+def test_long_sequence_sampled():
+    # N = 65536 keys per head: 256 work tiles of one head pair, 512 key blocks each
+    q, k, v = synth.random_inputs(1, 2, 65536, 64, BF16, seed=81)
+    o, lse = run_fwd(q, k, v, False)
+    rows = [0, 1, 127, 128, 255, 256, 40000, 65535]
+    check(o, lse, q, k, v, fa.default_scale(64), False, rows=rows, label="N=65536")
+    o, lse = run_fwd(q, k, v, True)
+    check(o, lse, q, k, v, fa.default_scale(64), True, rows=rows, label="N=65536 causal")
+
+
+def test_many_heads_short_sequence():
+    # 4096 (b, h) problems of 96 rows: one partly filled Q tile each
+    q, k, v = synth.random_inputs(64, 64, 96, 128, FP16, seed=91)
+    o, lse = run_fwd(q, k, v, True)
+    O, L = oracle.attention(q[:2], k[:2], v[:2], scale=fa.default_scale(128), causal=True)
+    import numpy as np
+    assert np.abs(o[:2].double().numpy() - O).max() <= 2e-2
+    # the remaining heads: closed-form property of the causal first row
+    assert torch.equal(o[:, :, 0], v[:, :, 0])
