@@ -51,8 +51,37 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         print(res.stderr)
+    check_register_split(res.stdout + res.stderr)
     os.replace(tmp, LIB)
     return LIB
+
+
+# The two-Q-tile kernels run 640 threads (96 registers each at launch) and
+# redistribute them with setmaxnreg: 4 * 128 * 104 + 128 * 64 = 61440.
+SPLIT_THREADS = 640
+SPLIT_REQUEST = 4 * 128 * 104 + 128 * 64
+
+
+def check_register_split(ptxas_log: str) -> None:
+    """Refuse a build whose setmaxnreg requests exceed the registers the
+    640-thread kernels are launched with: such a request would never be
+    granted and the kernel would wait for it forever."""
+    import re
+    entry, seen = None, 0
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '(\S+)'", line)
+        if m:
+            entry = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and entry and re.search(r"fa_fwd_kernelILi\d+ELi2E", entry):
+            regs = int(m.group(1))
+            if regs * SPLIT_THREADS < SPLIT_REQUEST:
+                raise RuntimeError(f"{entry}: {regs} registers x {SPLIT_THREADS} threads < "
+                                   f"setmaxnreg requests {SPLIT_REQUEST}")
+            seen += 1
+    if seen == 0:
+        raise RuntimeError("ptxas register report for the two-Q-tile kernels not found")
 
 
 if __name__ == "__main__":

@@ -17,18 +17,21 @@
 //   * one thread of the MMA warp issues tcgen05 MMAs: S = Q K^T into tensor
 //     memory (TMEM) and O += P V, both from shared-memory operands, committing
 //     each group to an mbarrier;
-//   * each softmax warpgroup owns one Q tile: thread t of the group owns query
-//     row t (TMEM lane t), so row max and row sum need no shuffles.  It reads
-//     S from TMEM and at once releases the S buffer, so the tensor core can
+//   * two softmax warpgroups own each Q tile, one per 64 key columns: thread t
+//     of a group owns query row t (TMEM lane t), so the row max and row sum
+//     need no shuffles, only one exchange per block between the two groups
+//     through shared memory.  Each group reads its half of S from TMEM and,
+//     once the row max is agreed, releases the S buffer so the tensor core can
 //     already compute the next block's S; then it applies scale (in the log2
-//     domain), the causal / ragged mask and the online update, writes P as
-//     16-bit values into shared memory in the layout the MMA reads, rescales O
-//     in TMEM when its reference max moved, and finally writes O / l and the
-//     logsumexp.
+//     domain), the causal / ragged mask and the online update, writes its
+//     half of P as 16-bit values into shared memory in the layout the MMA
+//     reads, rescales its half of O in TMEM when the reference max moved, and
+//     finally writes its half of O / l and (one group) the logsumexp.
 //
 // Because S(j+1) is computed while the softmax of block j runs, the softmax
-// groups work back to back and the two of them overlap on every SM
-// sub-partition, which one warp alone cannot do for the exponential unit.
+// groups work back to back; four of them share each SM sub-partition, which
+// hides the latency of the TMEM loads, the exponential unit and the hand-off
+// fences that two alone leave exposed.
 //
 // The running max used as the exp2 reference is only moved when the block max
 // exceeds it by more than 2^8 (in log2 units 8): O, l and the reference stay
@@ -62,7 +65,7 @@ __device__ unsigned int g_fa_watchdog = 0u;
 
 enum WaitSite : unsigned {
   kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteODone,
-  kSiteSelfTest, kSiteDrain, kSiteSFree, kSitePFree
+  kSiteSelfTest, kSiteDrain, kSiteSFree, kSitePFree, kSiteAlign, kSiteXch
 };
 enum Role : unsigned { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4 };
 
@@ -108,12 +111,20 @@ struct FwdCfg {
   static constexpr int CHUNK_BYTES = 128 * 128;   // one chunk of a 128-row tile
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
   static constexpr int P_TILE_BYTES = (BN / 64) * CHUNK_BYTES;  // 128 x 128 16-bit P
-  static constexpr int SOFTMAX_WARPS = 4 * QS;
+  // two softmax warpgroups per Q tile: key columns 0-63 and 64-127 of the
+  // same 128 rows
+  static constexpr int SOFTMAX_WGS = 2 * QS;
+  static constexpr int SOFTMAX_WARPS = 4 * SOFTMAX_WGS;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
   static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
   // whole warpgroups: the softmax groups, then one group holding the producer
   // warp, the MMA warp and two warps without a role
-  static constexpr int THREADS = 128 * (QS + 1);
+  static constexpr int THREADS = 128 * (SOFTMAX_WGS + 1);
+  // With 640 threads the launch budget is 96 registers a thread; setmaxnreg
+  // moves registers from the last warpgroup to the softmax groups:
+  // 4 * 128 * 104 + 128 * 64 = 61440 = 640 * 96 (the build checks the 96).
+  static constexpr bool REG_SPLIT = THREADS == 640;
+  static constexpr int SOFTMAX_REGS = 104, OTHER_REGS = 64;
 
   static constexpr int SQ_OFF = 0;
   static constexpr int SP_OFF = QS * TILE_BYTES;
@@ -124,10 +135,15 @@ struct FwdCfg {
                        B_S_FULL = 2 + 2 * KVS, B_S_FREE = B_S_FULL + 2,
                        B_P_FULL = B_S_FREE + 2,  // [Q tile][half of P]
                        B_P_FREE = B_P_FULL + 4, B_O_FINAL = B_P_FREE + 2,
-                       B_DRAIN = B_O_FINAL + 2, NUM_BARS = B_DRAIN + 1;
+                       B_XCH = B_O_FINAL + 2,  // the two softmax groups of a tile met
+                       B_DRAIN = B_XCH + 2, NUM_BARS = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack for 1024-B alignment
-  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static constexpr int XCH_OFF = MISC_OFF + 16;  // row max / row sum exchange [tile][half][row]
+  static constexpr int END_OFF = XCH_OFF + 2 * 2 * 128 * 4;
+  static_assert(END_OFF <= 232448, "shared memory budget");
+  // whatever is left up to the 227 KB limit pads the start to 1024 bytes
+  static constexpr int ALIGN_SLACK = (232448 - END_OFF) < 1008 ? (232448 - END_OFF) : 1008;
+  static constexpr int SMEM_BYTES = END_OFF + ALIGN_SLACK;
 
   // TMEM columns (fp32 words): one S buffer per Q tile, then the O accumulators.
   static constexpr uint32_t TMEM_COLS = 512;
@@ -419,20 +435,17 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return r;
 }
 
-// Max of 128 scores as a balanced tree of 3-input maxima.
-__device__ __forceinline__ float row_max128(const float* sv) {
-  float t[43];
+// Max of 64 scores as a balanced tree of 3-input maxima.
+__device__ __forceinline__ float row_max64(const float* sv) {
+  float t[22];
 #pragma unroll
-  for (int i = 0; i < 42; ++i) t[i] = max3(sv[3 * i], sv[3 * i + 1], sv[3 * i + 2]);
-  t[42] = fmaxf(sv[126], sv[127]);
-  float u[15];
+  for (int i = 0; i < 21; ++i) t[i] = max3(sv[3 * i], sv[3 * i + 1], sv[3 * i + 2]);
+  t[21] = sv[63];
+  float u[8];
 #pragma unroll
-  for (int i = 0; i < 14; ++i) u[i] = max3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
-  u[14] = t[42];
-  float v[5];
-#pragma unroll
-  for (int i = 0; i < 5; ++i) v[i] = max3(u[3 * i], u[3 * i + 1], u[3 * i + 2]);
-  return fmaxf(max3(v[0], v[1], v[2]), fmaxf(v[3], v[4]));
+  for (int i = 0; i < 7; ++i) u[i] = max3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+  u[7] = t[21];
+  return fmaxf(max3(u[0], u[1], u[2]), max3(u[3], u[4], fmaxf(u[5], fmaxf(u[6], u[7]))));
 }
 
 // Writes 64 keys of one P row (32 packed pairs) into the 128-byte swizzled,
@@ -474,19 +487,36 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
                              volatile int* abort_flag) {
   using C = FwdCfg<HD, QS, KVS, BF16>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  constexpr int HD2 = HD / 2;                 // O columns each group of a tile owns
   const uint32_t bars = base + C::BAR_OFF;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int s = warp / 4;                   // which Q tile of the work tile
-  const int r = (warp % 4) * 32 + lane;     // query row within the tile == TMEM lane
+  const int wg = warp / 4;
+  const int s = wg >> 1;                      // which Q tile of the work tile
+  const int hf = wg & 1;                      // which 64 key columns of its S rows
+  const int r = (warp % 4) * 32 + lane;       // query row within the tile == TMEM lane
   const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp % 4) * 32u) << 16);
-  const uint32_t s_col = C::s_col(s);
-  const uint32_t o_col = s ? C::O_COL1 : C::O_COL0;
-  const uint32_t sp = base + C::SP_OFF + s * C::P_TILE_BYTES;
+  const uint32_t s_col = C::s_col(s) + 64u * hf;
+  const uint32_t o_col = (s ? C::O_COL1 : C::O_COL0) + HD2 * hf;
+  const uint32_t sp = base + C::SP_OFF + s * C::P_TILE_BYTES + hf * C::CHUNK_BYTES;
+  float* xch = reinterpret_cast<float*>(
+      __cvta_shared_to_generic(base + C::XCH_OFF));
+  float* x_mine = xch + (s * 2 + hf) * 128;
+  const float* x_other = xch + (s * 2 + (hf ^ 1)) * 128;
   const unsigned long long lim = p.wait_limit_ns;
   const float sl2 = p.scale_log2;
   const int G = gridDim.x, cta = blockIdx.x;
-  uint32_t s_par = 0u, pf_par = 0u, fin_par = 0u;
+  uint32_t s_par = 0u, pf_par = 0u, fin_par = 0u, x_par = 0u;
   int p_written = 0;  // P blocks this Q tile has handed to the MMA warp so far
+  // Both softmax groups of the tile arrive (one arrival per warp, after the
+  // warp's shared-memory writes) and wait for each other, with the bounded wait.
+  auto group_meet = [&]() -> bool {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars + 8 * (C::B_XCH + s));
+    const bool met = wait_phase(bars + 8 * (C::B_XCH + s), x_par, abort_flag, lim,
+                                (kRoleSoftmax << 8) | kSiteXch);
+    x_par ^= 1u;
+    return __all_sync(0xffffffffu, met);
+  };
 
   for (int round = 0; round * G < p.num_tiles; ++round) {
     const int t = tile_of(round, cta, G);
@@ -507,26 +537,33 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       s_par ^= 1u;
       if (!__all_sync(0xffffffffu, ok)) return;
       tc_fence_after_sync();
-      uint32_t sr[128];
-      tmem_ld128_sync(lane_base + s_col, sr);
-      // S is in registers: the MMA warp may overwrite the buffer with S(j+1).
+      uint32_t sr[64];
+      tmem_ld64_nowait(lane_base + s_col, sr);
+      tmem_ld64_wait(sr);
+      float sv[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c]);
+      const bool need_mask = j >= first_masked;
+      if (need_mask) {
+        const int lim_local = limit - j * BN - 64 * hf;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sv[c] = (c < lim_local) ? sv[c] : -INFINITY;
+      }
+      // row max over both halves of the row
+      const float m_half = row_max64(sv) * sl2;
+      x_mine[r] = m_half;
+      if (!group_meet()) return;
+      const float m_blk = fmaxf(m_half, x_other[r]);
+      // S is in registers and both groups have read the exchange slot: the MMA
+      // warp may overwrite the S buffer with S(j+1), and the slots are free
+      // again once that S arrives.
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8 * (C::B_S_FREE + s));
 
-      float sv[128];
-#pragma unroll
-      for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-      const bool need_mask = j >= first_masked;
-      if (need_mask) {
-        const int lim_local = limit - j * BN;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = (c < lim_local) ? sv[c] : -INFINITY;
-      }
-      const float m_blk = row_max128(sv) * sl2;
-
       // Lazy reference: keep m_ref unless the block max exceeds it by more
-      // than 2^8; the first block always sets it.
+      // than 2^8; the first block always sets it.  Both groups of the tile
+      // take the same decision from the same values.
       const bool rescale = (j > 0) && (m_blk > m_ref + kLazyRescaleLog2);
       const float m_new = (j == 0 || rescale) ? m_blk : m_ref;
       const float alpha = (j == 0) ? 0.f : ex2(m_ref - m_new);  // 1 when m_ref is kept
@@ -535,61 +572,60 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
 
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
+      uint32_t pk[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (need_mask)
-            softmax_chunk<BF16, 0>(sv + 64 * half + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
-          else
-            softmax_chunk<BF16, kPolyPairsPer8>(sv + 64 * half + 32 * c, sl2, neg_ref,
-                                                pk + 16 * c, acc);
-        }
-        if (half == 0) {
-          // The previous P V has finished: its P buffer is free and O holds it.
-          if (p_written > 0) {
-            ok = wait_phase(bars + 8 * (C::B_P_FREE + s), pf_par, abort_flag, lim,
-                            (kRoleSoftmax << 8) | kSitePFree);
-            pf_par ^= 1u;
-            if (!__all_sync(0xffffffffu, ok)) return;
-            tc_fence_after_sync();
-          }
-          if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll 1
-            for (int c = 0; c < HD; c += 16) {
-              uint32_t ov[16];
-              tmem_ld16_sync(lane_base + o_col + c, ov);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-              tmem_st16(lane_base + o_col + c, ov);
-            }
-            tmem_st_wait();
-          }
-        }
-        store_p_chunk(sp + half * C::CHUNK_BYTES, r, pk);
-        // make the generic-proxy stores visible to the tensor core
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + 2 * s + half));
+      for (int c = 0; c < 2; ++c) {
+        if (need_mask)
+          softmax_chunk<BF16, 0>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
+        else
+          softmax_chunk<BF16, kPolyPairsPer8>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
       }
+      // The previous P V has finished: its P buffer is free and O holds it.
+      if (p_written > 0) {
+        ok = wait_phase(bars + 8 * (C::B_P_FREE + s), pf_par, abort_flag, lim,
+                        (kRoleSoftmax << 8) | kSitePFree);
+        pf_par ^= 1u;
+        if (!__all_sync(0xffffffffu, ok)) return;
+        tc_fence_after_sync();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll 1
+        for (int c = 0; c < HD2; c += 16) {
+          uint32_t ov[16];
+          tmem_ld16_sync(lane_base + o_col + c, ov);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st16(lane_base + o_col + c, ov);
+        }
+        tmem_st_wait();
+      }
+      store_p_chunk(sp, r, pk);
+      // make the generic-proxy stores visible to the tensor core
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + 2 * s + hf));
       ++p_written;
       const float2 acc01 = __fadd2_rn(acc[0], acc[1]), acc23 = __fadd2_rn(acc[2], acc[3]);
       l = l * alpha + ((acc01.x + acc23.x) + (acc01.y + acc23.y));
     }
 
-    // Epilogue: wait for the last P V product, then O / l and the logsumexp.
+    // Epilogue: wait for the last P V product; each group writes its half of
+    // the O columns, divided by the row sum of both halves.
     bool ok = wait_phase(bars + 8 * (C::B_O_FINAL + s), fin_par, abort_flag, lim,
                          (kRoleSoftmax << 8) | kSiteODone);
     fin_par ^= 1u;
     if (!__all_sync(0xffffffffu, ok)) return;
     tc_fence_after_sync();
-    const float inv_l = 1.f / l;
+    x_mine[r] = l;
+    if (!group_meet()) return;
+    const float l_row = l + x_other[r];
+    if (!group_meet()) return;  // both have read before the slots are reused
+    const float inv_l = 1.f / l_row;
     T* orow = reinterpret_cast<T*>(p.o) + ti.b * p.o_stride_b + ti.h * p.o_stride_h +
-              static_cast<long long>(row) * p.o_stride_n;
+              static_cast<long long>(row) * p.o_stride_n + HD2 * hf;
 #pragma unroll 1
-    for (int c = 0; c < HD; c += 32) {
+    for (int c = 0; c < HD2; c += 32) {
       uint32_t ov[32];
       tmem_ld32_sync(lane_base + o_col + c, ov);
       uint4 w[4];
@@ -603,9 +639,9 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         for (int i = 0; i < 4; ++i) dst[i] = w[i];
       }
     }
-    if (p.lse != nullptr && row < p.N)
+    if (hf == 0 && p.lse != nullptr && row < p.N)
       p.lse[(static_cast<long long>(ti.b) * p.H + ti.h) * p.N + row] =
-          (m_ref + log2f(l)) * 0.69314718055994530942f;
+          (m_ref + log2f(l_row)) * 0.69314718055994530942f;
     // The next tile's first P V overwrites O only after this group's next
     // P arrival, which comes after these loads completed.
     tc_fence_before_sync();
@@ -619,6 +655,11 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
+  if (base - raw > static_cast<uint32_t>(C::ALIGN_SLACK)) {
+    // the 1024-byte-aligned layout would not fit the allocation: refuse
+    if (threadIdx.x == 0) atomicCAS(&g_fa_watchdog, 0u, (kRoleTest << 8) | kSiteAlign);
+    return;
+  }
   uint8_t* smem = smem_raw + (base - raw);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
@@ -633,8 +674,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
       mbar_init(bars + 8 * (C::B_KV_EMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + 8 * (C::B_XCH + i), 8);  // one arrival per softmax warp of the tile
       mbar_init(bars + 8 * (C::B_S_FULL + i), 1);
-      mbar_init(bars + 8 * (C::B_S_FREE + i), 4);  // one arrival per softmax warp
+      mbar_init(bars + 8 * (C::B_S_FREE + i), 8);  // one arrival per softmax warp of the tile
       mbar_init(bars + 8 * (C::B_P_FREE + i), 1);
       mbar_init(bars + 8 * (C::B_O_FINAL + i), 1);
     }
@@ -656,6 +698,13 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_holder;
+
+  if constexpr (C::REG_SPLIT) {
+    if (warp < C::SOFTMAX_WARPS)
+      reg_alloc<C::SOFTMAX_REGS>();
+    else
+      reg_dealloc<C::OTHER_REGS>();
+  }
 
   if (warp < C::SOFTMAX_WARPS) {
     softmax_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
