@@ -17,7 +17,11 @@ namespace {
 using namespace fa_sm100;
 
 constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per mbarrier wait
+// Limit of every mbarrier wait of the kernel (2 s unless the build sets it).
+#ifndef FA_WAIT_LIMIT_NS
+#define FA_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = FA_WAIT_LIMIT_NS;
 constexpr int kMaxDevices = 64;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -92,8 +96,8 @@ int encode_operand(CUtensorMap* map, const void* ptr, int dtype, int d, int N, i
 
 // Kernel configuration per head dim: (Q tiles per work tile, K/V ring stages).
 template <int HD> struct Pick;
-template <> struct Pick<64> { static constexpr int QS = 2, KVS = 8; };
-template <> struct Pick<128> { static constexpr int QS = 2, KVS = 3; };
+template <> struct Pick<64> { static constexpr int QS = 2, KVS = 10; };
+template <> struct Pick<128> { static constexpr int QS = 2, KVS = 4; };
 template <> struct Pick<256> { static constexpr int QS = 1, KVS = 2; };
 
 int q_tiles_for(int d) { return d == 256 ? 1 : 2; }

@@ -64,8 +64,9 @@ constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;
 __device__ unsigned int g_fa_watchdog = 0u;
 
 enum WaitSite : unsigned {
-  kSiteQEmpty = 1, kSiteKvEmpty, kSiteQFull, kSiteKvFull, kSitePFull, kSiteSFull, kSiteODone,
-  kSiteSelfTest, kSiteDrain, kSiteSFree, kSitePFree, kSiteAlign, kSiteXch
+  kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteQFull = 3, kSiteKvFull = 4, kSitePFull = 5,
+  kSiteSFull = 6, kSiteODone = 7, kSiteSelfTest = 8, kSiteDrain = 9, kSiteSFree = 10,
+  kSitePFree = 11, kSiteAlign = 12, kSiteXch = 13
 };
 enum Role : unsigned { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4 };
 
@@ -110,15 +111,17 @@ struct FwdCfg {
   static constexpr int CHUNKS = HD / 64;          // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = 128 * 128;   // one chunk of a 128-row tile
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
-  static constexpr int P_TILE_BYTES = (BN / 64) * CHUNK_BYTES;  // 128 x 128 16-bit P
+  // one 128 x 128 16-bit P tile, used by the Q tiles in turn
+  static constexpr int P_TILE_BYTES = (BN / 64) * CHUNK_BYTES;
   // two softmax warpgroups per Q tile: key columns 0-63 and 64-127 of the
   // same 128 rows
   static constexpr int SOFTMAX_WGS = 2 * QS;
   static constexpr int SOFTMAX_WARPS = 4 * SOFTMAX_WGS;
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
-  static constexpr int MMA_WARP = SOFTMAX_WARPS + 1;
+  static constexpr int MMA_S_WARP = SOFTMAX_WARPS + 1;   // issues S = Q K^T, owns TMEM
+  static constexpr int MMA_PV_WARP = SOFTMAX_WARPS + 2;  // issues O += P V
   // whole warpgroups: the softmax groups, then one group holding the producer
-  // warp, the MMA warp and two warps without a role
+  // warp, the two MMA warps and one warp without a role
   static constexpr int THREADS = 128 * (SOFTMAX_WGS + 1);
   // With 640 threads the launch budget is 96 registers a thread; setmaxnreg
   // moves registers from the last warpgroup to the softmax groups:
@@ -128,15 +131,18 @@ struct FwdCfg {
 
   static constexpr int SQ_OFF = 0;
   static constexpr int SP_OFF = QS * TILE_BYTES;
-  static constexpr int SKV_OFF = SP_OFF + QS * P_TILE_BYTES;
+  static constexpr int SKV_OFF = SP_OFF + P_TILE_BYTES;
   static constexpr int BAR_OFF = SKV_OFF + KVS * TILE_BYTES;
   // barrier indices ([Q tile] unless noted)
   static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_KV_FULL = 2, B_KV_EMPTY = 2 + KVS,
                        B_S_FULL = 2 + 2 * KVS, B_S_FREE = B_S_FULL + 2,
-                       B_P_FULL = B_S_FREE + 2,  // [Q tile][half of P]
-                       B_P_FREE = B_P_FULL + 4, B_O_FINAL = B_P_FREE + 2,
+                       B_P_FULL = B_S_FREE + 2,  // [half of P] of the tile using the buffer
+                       B_P_FREE = B_P_FULL + 2,  // [Q tile][half]: that half is this tile's turn
+                       B_PV_DONE = B_P_FREE + 4,  // [Q tile]: a P V product of the tile finished
+                       B_O_FINAL = B_PV_DONE + 2,
                        B_XCH = B_O_FINAL + 2,  // the two softmax groups of a tile met
-                       B_DRAIN = B_XCH + 2, NUM_BARS = B_DRAIN + 1;
+                       B_DRAIN = B_XCH + 2,    // [MMA thread]
+                       NUM_BARS = B_DRAIN + 2;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int XCH_OFF = MISC_OFF + 16;  // row max / row sum exchange [tile][half][row]
   static constexpr int END_OFF = XCH_OFF + 2 * 2 * 128 * 4;
@@ -191,10 +197,20 @@ __device__ __forceinline__ TileInfo decode_tile(const FwdParams& p, int t) {
   return ti;
 }
 
-// Ring positions (from the work tile's first) of K(j) and V(j) when a work
-// tile streams K(0), then K(j+1), V(j) for j = 0 .. n-2, then V(n-1).
-__host__ __device__ __forceinline__ int ring_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
-__host__ __device__ __forceinline__ int ring_v(int j, int n) { return j < n - 1 ? 2 * j + 2 : 2 * n - 1; }
+// Ring positions (from the work tile's first) of K(j) and V(j): a work tile
+// streams K(0), V(0), K(1), V(1), ...
+__host__ __device__ __forceinline__ int ring_k(int j) { return 2 * j; }
+__host__ __device__ __forceinline__ int ring_v(int j) { return 2 * j + 1; }
+
+// Order in which the Q tiles of a work tile use the shared P buffer: block j
+// of tile 0, then block j of tile 1, then block j + 1 of tile 0, ...  Returns
+// the tile of the use after (s, j), or -1 if (s, j) is the work tile's last.
+__device__ __forceinline__ int next_p_user(int s, int j, const int (&n)[2]) {
+  if (s == 0 && j < n[1]) return 1;
+  if (j + 1 < n[0]) return 0;
+  if (j + 1 < n[1]) return 1;
+  return -1;
+}
 
 // Static persistent schedule: round r hands tiles [r*G, (r+1)*G) to the G
 // CTAs, reversing the order on odd rounds, so that with the longest-first
@@ -260,9 +276,8 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
         tma_load_4d(base + C::SQ_OFF + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tmap_q,
                     bars + 8 * C::B_Q_FULL, c * 64, ti.q0 + s * BM, ti.h, ti.b);
     ++q_count;
-    ok = load_kv(&p.tmap_k, 0, ti);
     for (int j = 0; ok && j < ti.n_max; ++j) {
-      if (j + 1 < ti.n_max && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
+      if (!(ok = load_kv(&p.tmap_k, j * BN, ti))) break;
       ok = load_kv(&p.tmap_v, j * BN, ti);
     }
   }
@@ -282,21 +297,24 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
   }
 }
 
-// Issue order per work tile (Q tile s = 0, 1; key block j):
-//   S_s(0)
-//   for each j:  S_s(j+1) once the softmax of tile s has read S_s(j),
-//                then P V_s(j) once it has written P_s(j).
+// The tensor core is fed by two threads, because a thread that issues
+// tcgen05.mma runs only about one instruction ahead of its execution: one
+// thread issues the S = Q K^T products, the other the O += P V products, so
+// that neither waits behind the other's dependencies.  Each commits only what
+// it issued.
+
+// S thread, per work tile: S_s(0) for every Q tile s, then S_s(j+1) once the
+// softmax of tile s has read S_s(j) out of TMEM.
 template <int HD, int QS, int KVS, bool BF16>
-__device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
-                         volatile int* abort_flag) {
+__device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
+                           volatile int* abort_flag) {
   using C = FwdCfg<HD, QS, KVS, BF16>;
   const uint32_t bars = base + C::BAR_OFF;
   const uint32_t idesc_qk = f16_idesc(BF16, BM, BN, false);
-  const uint32_t idesc_pv = f16_idesc(BF16, BM, HD, true);
   const unsigned long long lim = p.wait_limit_ns;
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0, q_count = 0;
-  uint32_t p_par[2] = {0u, 0u}, sf_par[2] = {0u, 0u};
+  uint32_t sf_par[2] = {0u, 0u};
   int s_issued[2] = {0, 0};
   bool ok = true;
 
@@ -329,30 +347,6 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     ++s_issued[s];
     return true;
   };
-  // O (+)= P V with P read from shared memory, handed over in two halves of
-  // 64 keys: the first four K-steps start once the first half is written.
-  auto issue_pv = [&](int s, int vslot, bool accumulate) -> bool {
-    const uint32_t pa = sw128_desc_lo(base + C::SP_OFF + s * C::P_TILE_BYTES, 16);
-    const uint32_t vb = sw128_desc_lo(base + C::SKV_OFF + vslot * C::TILE_BYTES, C::CHUNK_BYTES);
-    const uint32_t d_tmem = tmem + (s ? C::O_COL1 : C::O_COL0);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      if (!wait_phase(bars + 8 * (C::B_P_FULL + 2 * s + half), p_par[s], abort_flag, lim,
-                      (kRoleMma << 8) | kSitePFull))
-        return false;
-      tc_fence_after_sync();
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int kk = half * 4 + k4;
-        mma_ss(d_tmem, desc_from_lo(pa + ((half * C::CHUNK_BYTES + k4 * 32) >> 4)),
-               desc_from_lo(vb + ((kk * 16 * 128) >> 4)), idesc_pv,
-               (accumulate || kk > 0) ? 1u : 0u);
-      }
-    }
-    p_par[s] ^= 1u;
-    tc_commit(bars + 8 * (C::B_P_FREE + s));
-    return true;
-  };
 
   for (int round = 0; ok && round * G < p.num_tiles; ++round) {
     const int t = tile_of(round, cta, G);
@@ -363,45 +357,100 @@ __device__ void mma_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     tc_fence_after_sync();
     ++q_count;
     if (!ok) break;
-    const int kv0 = kv_count, n_max = ti.n_max;
-    // S(0)
-    if (!(ok = wait_kv(kv0 + ring_k(0)))) break;
-#pragma unroll
-    for (int s = 0; s < QS; ++s)
-      if (ok && ti.n[s] > 0) ok = issue_s(s, (kv0 + ring_k(0)) % KVS);
-    if (!ok) break;
-    tc_commit(bars + 8 * (C::B_KV_EMPTY + (kv0 + ring_k(0)) % KVS));
-    if (n_max == 1) tc_commit(bars + 8 * C::B_Q_EMPTY);
-    for (int j = 0; ok && j < n_max; ++j) {
-      if (j + 1 < n_max) {  // S(j+1)
-        const int k_idx = kv0 + ring_k(j + 1);
-        if (!(ok = wait_kv(k_idx))) break;
-#pragma unroll
-        for (int s = 0; s < QS; ++s)
-          if (ok && j + 1 < ti.n[s]) ok = issue_s(s, k_idx % KVS);
-        if (!ok) break;
-        tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
-        if (j + 2 == n_max) tc_commit(bars + 8 * C::B_Q_EMPTY);
-      }
-      // P V(j)
-      const int v_idx = kv0 + ring_v(j, n_max);
-      if (!(ok = wait_kv(v_idx))) break;
-#pragma unroll
+    const int kv0 = kv_count;
+    for (int j = 0; ok && j < ti.n_max; ++j) {
+      const int k_idx = kv0 + ring_k(j);
+      if (!(ok = wait_kv(k_idx))) break;
+#pragma unroll 1
       for (int s = 0; s < QS; ++s)
-        if (ok && j < ti.n[s]) {
-          ok = issue_pv(s, v_idx % KVS, j > 0);
-          if (ok && j == ti.n[s] - 1) tc_commit(bars + 8 * (C::B_O_FINAL + s));
-        }
+        if (ok && j < ti.n[s]) ok = issue_s(s, k_idx % KVS);
       if (!ok) break;
-      tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
+      tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
+      if (j + 1 == ti.n_max) tc_commit(bars + 8 * C::B_Q_EMPTY);
     }
-    kv_count = kv0 + 2 * n_max;
+    kv_count = kv0 + 2 * ti.n_max;
   }
   if (!ok) {
     // Wait for every MMA this thread issued before TMEM is released.
     volatile int no_abort = 0;
     tc_commit(bars + 8 * C::B_DRAIN);
     wait_phase(bars + 8 * C::B_DRAIN, 0, &no_abort, 10000000ull, (kRoleMma << 8) | kSiteDrain);
+  }
+}
+
+// P V thread, per work tile and key block j: O_s (+)= P_s(j) V(j) for tile 0
+// then tile 1, each once the softmax has written P_s(j) into the shared P
+// buffer; after each product the buffer is handed to the tile that uses it
+// next (which also tells that tile's softmax that O_s holds the product).
+template <int HD, int QS, int KVS, bool BF16>
+__device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
+                            volatile int* abort_flag) {
+  using C = FwdCfg<HD, QS, KVS, BF16>;
+  const uint32_t bars = base + C::BAR_OFF;
+  const uint32_t idesc_pv = f16_idesc(BF16, BM, HD, true);
+  const unsigned long long lim = p.wait_limit_ns;
+  const int G = gridDim.x, cta = blockIdx.x;
+  int kv_count = 0;
+  uint32_t p_par = 0u;
+  bool ok = true;
+  const uint32_t pa = sw128_desc_lo(base + C::SP_OFF, 16);
+
+  // O (+)= P V with P read from shared memory, handed over in two halves of
+  // 64 keys: the first four K-steps start once the first half is written and
+  // both halves of O are rescaled.  Once a half's K-steps have run, that half
+  // of the buffer goes to the next user (tile `nxt`).
+  auto issue_pv = [&](int s, int vslot, bool accumulate, int nxt) -> bool {
+    const uint32_t vb = sw128_desc_lo(base + C::SKV_OFF + vslot * C::TILE_BYTES, C::CHUNK_BYTES);
+    const uint32_t d_tmem = tmem + (s ? C::O_COL1 : C::O_COL0);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      if (!wait_phase(bars + 8 * (C::B_P_FULL + half), p_par, abort_flag, lim,
+                      (kRoleMma << 8) | kSitePFull))
+        return false;
+      tc_fence_after_sync();
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = half * 4 + k4;
+        mma_ss(d_tmem, desc_from_lo(pa + ((half * C::CHUNK_BYTES + k4 * 32) >> 4)),
+               desc_from_lo(vb + ((kk * 16 * 128) >> 4)), idesc_pv,
+               (accumulate || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(bars + 8 * (C::B_P_FREE + 2 * nxt + half));
+    }
+    tc_commit(bars + 8 * (C::B_PV_DONE + s));
+    p_par ^= 1u;
+    return true;
+  };
+
+  for (int round = 0; ok && round * G < p.num_tiles; ++round) {
+    const int t = tile_of(round, cta, G);
+    if (t >= p.num_tiles) continue;
+    const TileInfo ti = decode_tile<QS>(p, t);
+    const int kv0 = kv_count;
+    for (int j = 0; ok && j < ti.n_max; ++j) {
+      const int v_idx = kv0 + ring_v(j);
+      ok = wait_phase(bars + 8 * (C::B_KV_FULL + v_idx % KVS), (v_idx / KVS) & 1, abort_flag, lim,
+                      (kRoleMma << 8) | kSiteKvFull);
+      tc_fence_after_sync();
+#pragma unroll 1
+      for (int s = 0; s < QS; ++s) {
+        if (!ok || j >= ti.n[s]) continue;
+        // the next work tile starts with tile 0
+        const int nxt = next_p_user(s, j, ti.n);
+        ok = issue_pv(s, v_idx % KVS, j > 0, nxt < 0 ? 0 : nxt);
+        if (!ok) break;
+        if (j == ti.n[s] - 1) tc_commit(bars + 8 * (C::B_O_FINAL + s));
+      }
+      if (!ok) break;
+      tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
+    }
+    kv_count = kv0 + 2 * ti.n_max;
+  }
+  if (!ok) {
+    volatile int no_abort = 0;
+    tc_commit(bars + 8 * (C::B_DRAIN + 1));
+    wait_phase(bars + 8 * (C::B_DRAIN + 1), 0, &no_abort, 10000000ull,
+               (kRoleMma << 8) | kSiteDrain);
   }
 }
 
@@ -497,7 +546,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp % 4) * 32u) << 16);
   const uint32_t s_col = C::s_col(s) + 64u * hf;
   const uint32_t o_col = (s ? C::O_COL1 : C::O_COL0) + HD2 * hf;
-  const uint32_t sp = base + C::SP_OFF + s * C::P_TILE_BYTES + hf * C::CHUNK_BYTES;
+  const uint32_t sp = base + C::SP_OFF + hf * C::CHUNK_BYTES;  // this group's half of P
   float* xch = reinterpret_cast<float*>(
       __cvta_shared_to_generic(base + C::XCH_OFF));
   float* x_mine = xch + (s * 2 + hf) * 128;
@@ -506,7 +555,10 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const float sl2 = p.scale_log2;
   const int G = gridDim.x, cta = blockIdx.x;
   uint32_t s_par = 0u, pf_par = 0u, fin_par = 0u, x_par = 0u;
-  int p_written = 0;  // P blocks this Q tile has handed to the MMA warp so far
+  int pv_count = 0;  // P V products of this Q tile issued before the current block
+  // The P buffer's first use in the kernel (tile 0, first block) has nothing
+  // to wait for; every later use waits for the buffer to be handed over.
+  bool first_use = s == 0;
   // Both softmax groups of the tile arrive (one arrival per warp, after the
   // warp's shared-memory writes) and wait for each other, with the bounded wait.
   auto group_meet = [&]() -> bool {
@@ -580,15 +632,25 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         else
           softmax_chunk<BF16, kPolyPairsPer8>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
       }
-      // The previous P V has finished: its P buffer is free and O holds it.
-      if (p_written > 0) {
-        ok = wait_phase(bars + 8 * (C::B_P_FREE + s), pf_par, abort_flag, lim,
+      // This group's half of the P buffer is this tile's turn: the previous
+      // user's K-steps that read it have run.
+      if (!first_use) {
+        ok = wait_phase(bars + 8 * (C::B_P_FREE + 2 * s + hf), pf_par, abort_flag, lim,
                         (kRoleSoftmax << 8) | kSitePFree);
         pf_par ^= 1u;
         if (!__all_sync(0xffffffffu, ok)) return;
         tc_fence_after_sync();
       }
+      first_use = false;
       if (__any_sync(0xffffffffu, rescale)) {
+        // O must hold P V_s(j-1) before it is rescaled.  Every earlier product
+        // of the tile is known to have finished (the buffer hand-overs came
+        // after them) and the next one needs this block's P, so the phase of
+        // P V_s(j-1) is the barrier's current or just completed one.
+        ok = wait_phase(bars + 8 * (C::B_PV_DONE + s), static_cast<uint32_t>(pv_count - 1) & 1u,
+                        abort_flag, lim, (kRoleSoftmax << 8) | kSitePFree);
+        if (!__all_sync(0xffffffffu, ok)) return;
+        tc_fence_after_sync();
 #pragma unroll 1
         for (int c = 0; c < HD2; c += 16) {
           uint32_t ov[16];
@@ -599,13 +661,20 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         }
         tmem_st_wait();
       }
+      // The first P V K-steps write all of O: the second group reports its
+      // half rescaled on the barrier of the first P half.
+      if (hf == 1) {
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * C::B_P_FULL);
+      }
       store_p_chunk(sp, r, pk);
       // make the generic-proxy stores visible to the tensor core
       fence_proxy_async_smem();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + 2 * s + hf));
-      ++p_written;
+      if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + hf));
+      ++pv_count;
       const float2 acc01 = __fadd2_rn(acc[0], acc[1]), acc23 = __fadd2_rn(acc[2], acc[3]);
       l = l * alpha + ((acc01.x + acc23.x) + (acc01.y + acc23.y));
     }
@@ -677,11 +746,16 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
       mbar_init(bars + 8 * (C::B_XCH + i), 8);  // one arrival per softmax warp of the tile
       mbar_init(bars + 8 * (C::B_S_FULL + i), 1);
       mbar_init(bars + 8 * (C::B_S_FREE + i), 8);  // one arrival per softmax warp of the tile
-      mbar_init(bars + 8 * (C::B_P_FREE + i), 1);
+      mbar_init(bars + 8 * (C::B_P_FREE + 2 * i), 1);
+      mbar_init(bars + 8 * (C::B_P_FREE + 2 * i + 1), 1);
+      mbar_init(bars + 8 * (C::B_PV_DONE + i), 1);
       mbar_init(bars + 8 * (C::B_O_FINAL + i), 1);
+      mbar_init(bars + 8 * (C::B_DRAIN + i), 1);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(bars + 8 * (C::B_P_FULL + i), 4);
-    mbar_init(bars + 8 * C::B_DRAIN, 1);
+    // first P half: the first group's warps once P is written and the second
+    // group's once their O half is rescaled; second half: the second group
+    mbar_init(bars + 8 * C::B_P_FULL, 8);
+    mbar_init(bars + 8 * (C::B_P_FULL + 1), 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -690,7 +764,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
     tma_prefetch_desc(&p.tmap_k);
     tma_prefetch_desc(&p.tmap_v);
   }
-  if (warp == C::MMA_WARP) {
+  if (warp == C::MMA_S_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -710,13 +784,15 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
     softmax_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
   } else if (warp == C::PRODUCER_WARP) {
     if (lane == 0) producer_role<HD, QS, KVS, BF16>(p, base, abort_flag);
-  } else if (warp == C::MMA_WARP) {
-    if (lane == 0) mma_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
-  }  // the remaining warps of the last warpgroup have no role
+  } else if (warp == C::MMA_S_WARP) {
+    if (lane == 0) mma_s_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
+  } else if (warp == C::MMA_PV_WARP) {
+    if (lane == 0) mma_pv_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
+  }  // the last warp has no role
 
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == C::MMA_WARP) {
+  if (warp == C::MMA_S_WARP) {
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem, C::TMEM_COLS);
