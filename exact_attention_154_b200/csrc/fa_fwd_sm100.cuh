@@ -53,11 +53,18 @@ namespace fa_sm100 {
 constexpr int BM = 128;  // query rows per Q tile (tcgen05 M)
 constexpr int BN = 128;  // key / value rows per K or V tile
 constexpr float kLazyRescaleLog2 = 8.0f;
-// Argument pairs (of every 8) whose exp2 runs on the FMA pipe instead of MUFU.
-#ifndef FA_POLY_PAIRS_PER8
-#define FA_POLY_PAIRS_PER8 2
+// Argument pairs (of every 8) whose exp2 runs on the FMA pipe instead of
+// MUFU.  With two Q tiles (d = 64, 128) the exponentials are cheaper on MUFU
+// alone; with one (d = 256) a quarter on the FMA pipe helps (measured).  A
+// build may fix the number for every head dim.
+template <int HD>
+__host__ __device__ constexpr int poly_pairs_per8() {
+#ifdef FA_POLY_PAIRS_PER8
+  return FA_POLY_PAIRS_PER8;
+#else
+  return HD == 256 ? 2 : 0;
 #endif
-constexpr int kPolyPairsPer8 = FA_POLY_PAIRS_PER8;
+}
 
 // Error word written by a kernel whose bounded wait ran out: 0 = none,
 // otherwise (role << 8) | site, first writer wins.
@@ -197,10 +204,12 @@ __device__ __forceinline__ TileInfo decode_tile(const FwdParams& p, int t) {
   return ti;
 }
 
-// Ring positions (from the work tile's first) of K(j) and V(j): a work tile
-// streams K(0), V(0), K(1), V(1), ...
-__host__ __device__ __forceinline__ int ring_k(int j) { return 2 * j; }
-__host__ __device__ __forceinline__ int ring_v(int j) { return 2 * j + 1; }
+// Ring positions (from the work tile's first) of K(j) and V(j) when a work
+// tile streams K(0), then K(j+1), V(j) for j = 0 .. n-2, then V(n-1): each K
+// tile is requested before the V tile of the block before it, so a K load
+// never queues behind a V slot that the slower P V has yet to release.
+__host__ __device__ __forceinline__ int ring_k(int j) { return j == 0 ? 0 : 2 * j - 1; }
+__host__ __device__ __forceinline__ int ring_v(int j, int n) { return j < n - 1 ? 2 * j + 2 : 2 * n - 1; }
 
 // Order in which the Q tiles of a work tile use the shared P buffer: block j
 // of tile 0, then block j of tile 1, then block j + 1 of tile 0, ...  Returns
@@ -276,8 +285,9 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
         tma_load_4d(base + C::SQ_OFF + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tmap_q,
                     bars + 8 * C::B_Q_FULL, c * 64, ti.q0 + s * BM, ti.h, ti.b);
     ++q_count;
+    ok = load_kv(&p.tmap_k, 0, ti);
     for (int j = 0; ok && j < ti.n_max; ++j) {
-      if (!(ok = load_kv(&p.tmap_k, j * BN, ti))) break;
+      if (j + 1 < ti.n_max && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
       ok = load_kv(&p.tmap_v, j * BN, ti);
     }
   }
@@ -428,7 +438,7 @@ __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const TileInfo ti = decode_tile<QS>(p, t);
     const int kv0 = kv_count;
     for (int j = 0; ok && j < ti.n_max; ++j) {
-      const int v_idx = kv0 + ring_v(j);
+      const int v_idx = kv0 + ring_v(j, ti.n_max);
       ok = wait_phase(bars + 8 * (C::B_KV_FULL + v_idx % KVS), (v_idx / KVS) & 1, abort_flag, lim,
                       (kRoleMma << 8) | kSiteKvFull);
       tc_fence_after_sync();
@@ -630,7 +640,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         if (need_mask)
           softmax_chunk<BF16, 0>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
         else
-          softmax_chunk<BF16, kPolyPairsPer8>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
+          softmax_chunk<BF16, poly_pairs_per8<HD>()>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
       }
       // This group's half of the P buffer is this tile's turn: the previous
       // user's K-steps that read it have run.
