@@ -272,6 +272,9 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
     const TileInfo ti = decode_tile<QS>(p, t);
+    // K(0) needs only a ring slot: request it before waiting for the previous
+    // work tile to release the Q buffer, so the two loads overlap.
+    if (!(ok = load_kv(&p.tmap_k, 0, ti))) break;
     if (q_count > 0) {
       ok = wait_phase(bars + 8 * C::B_Q_EMPTY, (q_count - 1) & 1, abort_flag, p.wait_limit_ns,
                       (kRoleProducer << 8) | kSiteQEmpty);
@@ -285,7 +288,6 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
         tma_load_4d(base + C::SQ_OFF + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tmap_q,
                     bars + 8 * C::B_Q_FULL, c * 64, ti.q0 + s * BM, ti.h, ti.b);
     ++q_count;
-    ok = load_kv(&p.tmap_k, 0, ti);
     for (int j = 0; ok && j < ti.n_max; ++j) {
       if (j + 1 < ti.n_max && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
       ok = load_kv(&p.tmap_v, j * BN, ti);
