@@ -17,9 +17,14 @@ Three independent implementations live here:
   extended with the causal mask and the logsumexp output.
 * :func:`oracle.brute.attention_fsum` -- a scalar pure-Python version using
   ``math.fsum`` for tiny inputs.
+* :func:`attention_bwd` -- the gradient of the plain definition with respect
+  to q, k, v (chain rule written out in ``fa_oracle.c``), pinned in
+  ``tests/test_oracle_bwd_pins.py`` by central finite differences of
+  :func:`attention`, closed forms and invariants.
 
 Parity status: every function here is pinned by tests in
-``tests/test_oracle_pins.py`` (closed forms, invariants, brute force and the
+``tests/test_oracle_pins.py`` and ``tests/test_oracle_bwd_pins.py`` (closed
+forms, invariants, brute force, finite differences and the
 recurrence-equals-definition check); none is "parity unpinned".
 """
 from __future__ import annotations
@@ -70,6 +75,10 @@ def _load():
                 dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
                 ctypes.c_int, dp]
             lib.oracle_attention_probs.restype = ctypes.c_int
+            lib.oracle_attention_bwd.argtypes = [
+                dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int]
+            lib.oracle_attention_bwd.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -130,6 +139,32 @@ def attention(q, k, v, scale: float | None = None, causal: bool = False,
     if rc != 0:
         raise ValueError(f"oracle_attention_fwd failed ({rc})")
     return o.reshape(lead + (nr, d)), lse.reshape(lead + (nr,))
+
+
+def attention_bwd(q, k, v, dout, scale: float | None = None, causal: bool = False):
+    """Gradient of :func:`attention`'s O with respect to q, k, v in fp64.
+
+    ``dout`` is the upstream gradient of O, shaped like ``q``.  Returns
+    ``(dQ, dK, dV)`` shaped like the inputs.  The chain rule through the same
+    plain definition (``oracle_attention_bwd`` in ``fa_oracle.c``).
+    """
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    if not (q.shape == k.shape == v.shape == dout.shape):
+        raise ValueError("q, k, v, dout must have the same shape")
+    shape = q.shape
+    N, d = shape[-2], shape[-1]
+    if q.ndim < 2 or q.ndim > 4:
+        raise ValueError("expected 2-D, 3-D or 4-D inputs")
+    heads = int(np.prod(shape[:-2])) if q.ndim > 2 else 1
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq, dk, dv = (np.empty(shape, dtype=np.float64) for _ in range(3))
+    rc = _load().oracle_attention_bwd(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(dout), _dptr(dq), _dptr(dk), _dptr(dv),
+        1, heads, N, d, float(scale), int(bool(causal)))
+    if rc != 0:
+        raise ValueError(f"oracle_attention_bwd failed ({rc})")
+    return dq, dk, dv
 
 
 def probs(q, k, i: int, scale: float | None = None, causal: bool = False):

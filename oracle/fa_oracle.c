@@ -1,5 +1,6 @@
 /*
- * fa_oracle.c -- fp64 CPU oracle for the exact attention forward.
+ * fa_oracle.c -- fp64 CPU oracle for the exact attention forward and its
+ * gradient (oracle_attention_bwd, at the end of this file).
  *
  * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
  * baseline leg of the benchmark may load this library.  The product path
@@ -136,6 +137,86 @@ int oracle_attention_probs(const double *q, const double *k, int N, int d,
     for (int j = 0; j < nvis; ++j) p_out[j] /= l;
     for (int j = nvis; j < N; ++j) p_out[j] = 0.0;
     return 0;
+}
+
+/*
+ * Gradient of the forward above with respect to q, k and v, for an upstream
+ * gradient dout of O (the logsumexp output is taken as not differentiated).
+ * The pages name the backward pass only by its recomputation of the score
+ * tile from saved row statistics ("Windows下RTX 3090编译Flash Attention 2.8.3
+ * 全指南", sections 1 and 7); what it computes is fixed by the forward
+ * definition and the chain rule, written out here per (b, h):
+ *
+ *   P[i,j]  = exp(s_ij - LSE_i)              visible keys, 0 elsewhere
+ *   dV[j]   = sum_i P[i,j] * dout[i]
+ *   dP[i,j] = dout[i] . v[j]
+ *   D_i     = sum_j P[i,j] * dP[i,j]
+ *   dS[i,j] = P[i,j] * (dP[i,j] - D_i)        (row softmax Jacobian)
+ *   dq[i]   = scale * sum_j dS[i,j] * k[j]
+ *   dk[j]   = scale * sum_i dS[i,j] * q[i]
+ *
+ * Layout as the forward: every array [B, H, N, d] row-major doubles.
+ * Returns 0 on success, -1 on a bad argument, -2 when out of memory.
+ */
+int oracle_attention_bwd(const double *q, const double *k, const double *v,
+                         const double *dout, double *dq, double *dk, double *dv,
+                         int B, int H, int N, int d, double scale, int causal)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    if (B < 1 || H < 1 || N < 1 || d < 1) return -1;
+    const long long heads = (long long)B * H;
+    int failed = 0;
+
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!p || !dp) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long long bh = 0; bh < heads; ++bh) {
+            if (!p || !dp) continue;
+            const size_t off = (size_t)bh * N * d;
+            const double *Q = q + off, *K = k + off, *V = v + off, *DO = dout + off;
+            double *DQ = dq + off, *DK = dk + off, *DV = dv + off;
+            memset(DQ, 0, sizeof(double) * (size_t)N * d);
+            memset(DK, 0, sizeof(double) * (size_t)N * d);
+            memset(DV, 0, sizeof(double) * (size_t)N * d);
+            for (int i = 0; i < N; ++i) {
+                const int nvis = visible_keys(i, N, causal);
+                const double *qrow = Q + (size_t)i * d;
+                const double *dorow = DO + (size_t)i * d;
+                double l;
+                row_weights(qrow, K, nvis, d, scale, p, &l);
+                for (int j = 0; j < nvis; ++j) p[j] /= l;
+                double D = 0.0;
+                for (int j = 0; j < nvis; ++j) {
+                    const double *vrow = V + (size_t)j * d;
+                    double dot = 0.0;
+                    for (int c = 0; c < d; ++c) dot += dorow[c] * vrow[c];
+                    dp[j] = dot;
+                    D += p[j] * dot;
+                }
+                double *dqrow = DQ + (size_t)i * d;
+                for (int j = 0; j < nvis; ++j) {
+                    const double ds = p[j] * (dp[j] - D);
+                    const double *krow = K + (size_t)j * d;
+                    double *dkrow = DK + (size_t)j * d;
+                    double *dvrow = DV + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqrow[c] += scale * ds * krow[c];
+                        dkrow[c] += scale * ds * qrow[c];
+                        dvrow[c] += p[j] * dorow[c];
+                    }
+                }
+            }
+        }
+        free(p);
+        free(dp);
+    }
+    return failed ? -2 : 0;
 }
 
 int oracle_num_threads(void)
