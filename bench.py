@@ -38,6 +38,7 @@ from exact_attention_154_b200 import dist as fdist  # noqa: E402
 from exact_attention_154_b200 import fa, synth  # noqa: E402
 
 METRIC = "attention fwd TFLOP/s (bf16, 1×B200) and % of dense tensor-core peak"
+METRIC_BWD = "attention bwd TFLOP/s (bf16, 1×B200), 10·N²·d per head (5·N²·d causal)"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fa_fwd_sm100_traffic.md")
@@ -368,6 +369,121 @@ def bench_gpu(args, w, key, world, rank, local):
     return line
 
 
+def bwd_inputs(w):
+    """q, k, v and a seeded upstream gradient dO, all [B, H, N, d], on the host."""
+    q, k, v = synth.make_inputs(w)
+    g = torch.Generator().manual_seed(w.seed + 500)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype)
+    return q, k, v, dout
+
+
+def bench_gpu_bwd(args, w, key, world, rank, local):
+    """One step = one fa_bwd call (row statistic, dK/dV and dQ kernels) on
+    inputs resident in HBM; O and LSE come from one forward beforehand."""
+    if w.layout != "bhnd" or w.d not in (64, 128):
+        raise SystemExit(f"--direction bwd needs a [B,H,N,d] workload with d in (64, 128): {key}")
+    w = fdist.shard_workload(w, world, rank)
+    host = bwd_inputs(w)
+    q, k, v, dout = (t.cuda() for t in host)
+    o, lse = fa.fwd(q, k, v, causal=w.causal)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    work = torch.empty((w.B, w.H, w.N), device="cuda", dtype=torch.float32)
+    lib = fa.load()
+    cargs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), work.data_ptr(), w.B, w.H, w.N, w.d, 0.0,
+             int(w.causal), w.dtype)
+
+    def go():
+        rc = lib.fa_bwd(*cargs, torch.cuda.current_stream().cuda_stream)
+        if rc:
+            raise fa.FaError(rc, "fa_bwd")
+
+    flops = 2.5 * w.flops
+    with ClockSampler(local) as clk:
+        ms = time_device(go, args.steps, args.warmup, world)
+    clocks = clk.summary()
+    # end to end: host q, k, v, O, LSE, dO in; dQ, dK, dV out, every step
+    pinned = [t.pin_memory() for t in host] + [o.cpu().pin_memory(), lse.cpu().pin_memory()]
+    outs = [torch.empty_like(t).pin_memory() for t in host[:3]]
+    devs = [torch.empty_like(t, device="cuda") for t in pinned]
+
+    def step():
+        for h_, d_ in zip(pinned, devs):
+            d_.copy_(h_, non_blocking=True)
+        grads = fa.bwd(devs[0], devs[1], devs[2], devs[4], devs[5], devs[3], causal=w.causal)
+        for g_, h_ in zip(grads, outs):
+            h_.copy_(g_, non_blocking=True)
+    e2e_steps = max(3, min(args.steps, 30))
+    for _ in range(3):
+        step()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    e2e_ms = dist_max(e0.elapsed_time(e1) / e2e_steps, world)
+    rc, detail = fa.device_status(clear=True)
+    if rc != fa.FA_OK:
+        raise RuntimeError(f"kernel watchdog fired ({detail:#x})")
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    e = 2
+    nd = w.B * w.H * w.N * w.d
+    line = {
+        "metric": METRIC_BWD, "value": round(world * achieved, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": synth.DTYPE_NAME[w.dtype], "data": "synthetic (seeded randn, see DESIGN.md)",
+        "config": dict(w.describe(), workload_key=key, direction="bwd",
+                       parallelism=f"replicas{world}" if world > 1 else "single-gpu",
+                       global_batch=w.B * world, seq_len=w.N,
+                       l2="inputs larger than L2" if 8 * nd * e > (126 << 20) else "inputs fit in L2"),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peaks["bf16_tflops"], "unit": UNIT,
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak_note": f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json)"
+                                  if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+                     "traffic": None,
+                     "algorithmic_bytes": 8 * nd * e + 12 * w.B * w.H * w.N,
+                     "kernel": "fa_bwd_kernel", "launches_per_step": 3},
+        "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pinned),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs),
+                "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if not clocks_ok(clocks):
+        line["clocks_rejected"] = True
+    return line, host
+
+
+def cpu_oracle_bwd_sample(w, host, target_s=12.0):
+    """The fp64 gradient oracle, as it stands, on the first heads of the
+    workload (it runs one (b, h) per host thread), sized to ~target_s."""
+    import oracle
+    oracle.build()
+    q, k, v, g = (t.double().numpy().reshape(w.B * w.H, w.N, w.d) for t in host)
+    scale = fa.default_scale(w.d)
+    t0 = time.perf_counter()
+    oracle.attention_bwd(q[:1], k[:1], v[:1], g[:1], scale=scale, causal=w.causal)
+    dt1 = max(time.perf_counter() - t0, 1e-4)
+    threads = oracle.num_threads()
+    heads = max(1, min(w.B * w.H, threads * max(1, int(target_s / dt1))))
+    t0 = time.perf_counter()
+    oracle.attention_bwd(q[:heads], k[:heads], v[:heads], g[:heads], scale=scale, causal=w.causal)
+    dt = time.perf_counter() - t0
+    fl = 2.5 * w.flops / (w.B * w.H) * heads
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "seconds": round(dt, 4),
+            "sample": f"{heads} of the {w.B * w.H} (b, h) heads of the workload, whole heads, "
+                      f"fp64 gradient oracle, one head per host thread"}
+
+
 def algorithmic_bytes(w):
     e = 2
     return 4 * w.B * w.H * w.N * w.d * e + 4 * w.B * w.H * w.N
@@ -382,6 +498,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads_by_key()))
     ap.add_argument("--sweep", action="store_true", help="one line per benchmark workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--direction", choices=["fwd", "bwd"], default="fwd",
+                    help="fwd: the forward (default); bwd: the gradient (fa_bwd)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -415,9 +533,16 @@ def main():
     keys = list(table) if args.sweep else [args.workload]
     for key in keys:
         w = table[key]
-        line = bench_gpu(args, w, key, world, rank, local)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.sweep:
-            line["cpu_baseline"] = cpu_oracle_sample(w)
+        if args.direction == "bwd":
+            if args.sweep and (w.layout != "bhnd" or w.d not in (64, 128)):
+                continue
+            line, host = bench_gpu_bwd(args, w, key, world, rank, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.sweep:
+                line["cpu_baseline"] = cpu_oracle_bwd_sample(w, host)
+        else:
+            line = bench_gpu(args, w, key, world, rank, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.sweep:
+                line["cpu_baseline"] = cpu_oracle_sample(w)
         if rank == 0:
             print(json.dumps(line), flush=True)
         torch.cuda.empty_cache()

@@ -10,7 +10,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
-#include "fa_fwd_sm100.cuh"
+#include "fa_bwd_sm100.cuh"
 
 namespace {
 
@@ -36,6 +36,7 @@ struct DeviceState {
   bool is_sm100 = false;
   int sm_count = 0;
   bool attr_set[6] = {false, false, false, false, false, false};
+  bool bwd_attr_set[8] = {false, false, false, false, false, false, false, false};
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -177,6 +178,33 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
   }
 }
 
+template <int HD, bool BF16, bool KV>
+int launch_bwd_kernel(const BwdParams& p, DeviceState& st, cudaStream_t stream) {
+  using C = BwdCfg<HD>;
+  auto kernel = fa_bwd_kernel<HD, BF16, KV>;
+  const int slot = (HD == 64 ? 0 : 4) + (BF16 ? 2 : 0) + (KV ? 1 : 0);
+  if (!st.bwd_attr_set[slot]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    st.bwd_attr_set[slot] = true;
+  }
+  kernel<<<p.B * p.H * p.nblk, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int HD, bool BF16>
+int launch_bwd(const BwdParams& p, DeviceState& st, cudaStream_t stream) {
+  const long long rows = (long long)p.B * p.H * p.N;
+  bwd_dsum_kernel<HD, BF16><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p.o, p.dout, p.dsum, rows);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  int rc = launch_bwd_kernel<HD, BF16, true>(p, st, stream);
+  if (rc != FA_OK) return rc;
+  return launch_bwd_kernel<HD, BF16, false>(p, st, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -208,6 +236,54 @@ int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int N, int H, 
   const long long sn = 3 * hd, sh = d, sb = (long long)N * 3 * hd;
   return run(base, base + 2 * hd, base + 4 * hd, o, lse, B, H, N, d, scale, causal, dtype, sn, sh,
              sb, hd, d, (long long)N * hd, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, float* workspace, int B, int H, int N,
+           int d, float scale, int causal, int dtype, struct CUstream_st* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_ARG;
+  int rc = check_common(B, H, N, d, &scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  for (const void* t : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
+                        static_cast<const void*>(dv)})
+    if (!aligned16(t)) return FA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
+    return FA_ERR_ALIGN;
+  const int nblk = (N + 127) / 128;
+  if ((long long)B * H * nblk > 0x7fffffffLL) return FA_ERR_ARG;
+
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if ((rc = get_encode_fn()) != FA_OK) return rc;
+  DeviceState* st = nullptr;
+  int dev = 0;
+  if ((rc = device_state(&st, &dev)) != FA_OK) return rc;
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  const long long sn = d, sh = (long long)N * d, sb = (long long)H * N * d;
+  if ((rc = encode_operand(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_operand(&p.tmap_do, dout, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dsum = workspace;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.causal = causal;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.nblk = nblk;
+  p.wait_limit_ns = kWaitLimitNs;
+  const bool bf16 = dtype == FA_BF16;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return bf16 ? launch_bwd<64, true>(p, *st, s) : launch_bwd<64, false>(p, *st, s);
+  return bf16 ? launch_bwd<128, true>(p, *st, s) : launch_bwd<128, false>(p, *st, s);
 }
 
 const char* fa_strerror(int status) {

@@ -1,0 +1,399 @@
+// fa_bwd_sm100.cuh -- attention backward (dQ, dK, dV) for sm_100a.
+//
+// Gradient of the forward in fa_fwd_sm100.cuh for an upstream gradient dO.
+// The score tile is recomputed from Q, K and the forward's per-row logsumexp
+// (the recomputation the pages describe for the backward pass of the
+// "Windows下RTX 3090编译Flash Attention 2.8.3全指南" page, sections 1 and 7);
+// everything else follows from the chain rule through the forward:
+//
+//   D_i     = sum_c dO[i,c] * O[i,c]                     (bwd_dsum_kernel)
+//   P[i,j]  = exp2(s_ij * scale * log2 e - LSE_i * log2 e)   visible keys
+//   dV[j]   = sum_i P[i,j] dO[i]
+//   dP[i,j] = dO[i] . V[j]
+//   dS[i,j] = P[i,j] (dP[i,j] - D_i)
+//   dK[j]   = scale * sum_i dS[i,j] Q[i]                 (bwd_dkdv_kernel)
+//   dQ[i]   = scale * sum_j dS[i,j] K[j]                 (bwd_dq_kernel)
+//
+// bwd_dkdv_kernel: one CTA per 128-key block j.  For every query block i it
+// computes S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM (tcgen05, SS),
+// forms P^T and dS^T in 16 bits in shared memory (one thread per key row),
+// and accumulates dV_j += P^T dO_i and dK_j += dS^T Q_i in TMEM.
+// bwd_dq_kernel: one CTA per 128-query block i; recomputes S and dP the same
+// way for every key block j and accumulates dQ_i += dS K_j in TMEM.
+//
+// Roles per CTA (192 threads): warps 0-3 compute P and dS (thread = TMEM
+// lane = tile row), warp 4 streams tiles with TMA, warp 5 owns TMEM and one of
+// its threads issues every tcgen05.mma.  Q/dO (resp. K/V) of the streamed
+// operand are single-buffered.  All mbarrier waits are bounded (wait_phase).
+#pragma once
+
+#include "fa_fwd_sm100.cuh"
+
+namespace fa_sm100 {
+
+struct BwdParams {
+  CUtensorMap tmap_q;   // 4-D (d, N, H, B) views, box 64 elements x 128 rows
+  CUtensorMap tmap_k;
+  CUtensorMap tmap_v;
+  CUtensorMap tmap_do;
+  const void* o;        // forward output [B, H, N, d]
+  const void* dout;     // upstream gradient [B, H, N, d]
+  const float* lse;     // forward logsumexp [B, H, N] (natural log)
+  float* dsum;          // workspace [B, H, N]: D_i
+  void* dq;             // outputs [B, H, N, d]
+  void* dk;
+  void* dv;
+  int B, H, N, causal;
+  float scale;
+  float scale_log2;     // scale * log2(e)
+  int nblk;             // 128-row blocks per (b, h)
+  unsigned long long wait_limit_ns;
+};
+
+template <int HD>
+struct BwdCfg {
+  static_assert(HD == 64 || HD == 128, "backward head dim");
+  static constexpr int CHUNKS = HD / 64;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;   // one [128 x HD] 16-bit tile
+  static constexpr int SQR_BYTES = 2 * CHUNK_BYTES;         // one [128 x 128] 16-bit tile
+  static constexpr int THREADS = 192;
+  static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
+  // shared memory: the two resident tiles, the two streamed tiles, the 16-bit
+  // P^T / dS^T tiles (dkdv) or dS tile (dq), two 128-float vectors, barriers
+  static constexpr int SA_OFF = 0;                           // K (dkdv) / Q (dq)
+  static constexpr int SB_OFF = TILE_BYTES;                  // V (dkdv) / dO (dq)
+  static constexpr int SC_OFF = 2 * TILE_BYTES;              // Q (dkdv) / K (dq)
+  static constexpr int SD_OFF = 3 * TILE_BYTES;              // dO (dkdv) / V (dq)
+  static constexpr int SP_OFF = 4 * TILE_BYTES;              // P^T (dkdv)
+  static constexpr int SDS_OFF = SP_OFF + SQR_BYTES;         // dS^T (dkdv) / dS (dq)
+  // per compute warp: lse*log2e [128] and D [128] of the streamed query block
+  static constexpr int VEC_OFF = SDS_OFF + SQR_BYTES;
+  static constexpr int BAR_OFF = VEC_OFF + 4 * 2 * 128 * 4;
+  static constexpr int B_RES_FULL = 0, B_STR_FULL = 1, B_STR_EMPTY = 2, B_SD_FULL = 3,
+                       B_PDS_FULL = 4, B_DONE = 5, B_DRAIN = 6, NUM_BARS = 7;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int END_OFF = MISC_OFF + 16;
+  static constexpr int SMEM_BYTES = END_OFF + 1024;  // + slack to align the base to 1024
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // TMEM columns: S (or S^T), dP (or dP^T), then the accumulators
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0_COL = 256, ACC1_COL = 256 + HD;
+};
+
+// D_i = dO_i . O_i in fp32, one warp per row.
+template <int HD, bool BF16>
+__global__ void __launch_bounds__(256) bwd_dsum_kernel(const void* __restrict__ o,
+                                                       const void* __restrict__ dout,
+                                                       float* __restrict__ dsum, long long rows) {
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  const T* orow = static_cast<const T*>(o) + row * HD;
+  const T* drow = static_cast<const T*>(dout) + row * HD;
+  float acc = 0.f;
+#pragma unroll
+  for (int c = lane; c < HD; c += 32) acc += static_cast<float>(orow[c]) * static_cast<float>(drow[c]);
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (lane == 0) dsum[row] = acc;
+}
+
+// 32 packed 16-bit pairs of one tile row into the 128-byte-swizzled K-major
+// layout the MMAs read (as store_p_chunk): row r of a 64-column chunk at
+// r * 128 bytes, its 16-byte group u at u ^ (r % 8).  `col0` is a multiple of
+// 32 in [0, 128): columns col0 .. col0 + 31.
+__device__ __forceinline__ void store_row32(uint32_t tile, int r, int col0, const uint32_t* pk) {
+  const uint32_t row = tile + static_cast<uint32_t>(col0 / 64) * (128u * 128u) +
+                       static_cast<uint32_t>(r) * 128u;
+  const uint32_t u0 = static_cast<uint32_t>((col0 % 64) / 8);
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    st_shared_v4(row + (((u0 + u) ^ (static_cast<uint32_t>(r) & 7u)) << 4), pk[4 * u],
+                 pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+}
+
+// Loads one [128 x HD] tile of a 4-D tensor map into shared memory.
+template <int HD>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                          int row0, int h, int b) {
+#pragma unroll
+  for (int c = 0; c < HD / 64; ++c)
+    tma_load_4d(dst + c * (128 * 128), map, bar, c * 64, row0, h, b);
+}
+
+// Writes 32 fp32 accumulator columns of one row (times `mul`) as 16-bit values.
+template <bool BF16>
+__device__ __forceinline__ void store_acc32(void* dst_row, const uint32_t* acc, float mul) {
+  uint4 w[4];
+  uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+    wp[i] = pack2<BF16>(__uint_as_float(acc[2 * i]) * mul, __uint_as_float(acc[2 * i + 1]) * mul);
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = w[i];
+}
+
+// KV = true: the dK/dV kernel (CTA per key block, streams Q and dO).
+// KV = false: the dQ kernel (CTA per query block, streams K and V).
+template <int HD, bool BF16, bool KV>
+__global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
+    fa_bwd_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  // this warp's copy of the per-column statistics (no cross-warp barrier, so
+  // a warp that leaves on an abandoned wait cannot strand the others)
+  float* lse2_s = reinterpret_cast<float*>(smem + C::VEC_OFF) + (threadIdx.x / 32 % 4) * 256;
+  float* dsum_s = lse2_s + 128;
+  const uint32_t bars = base + C::BAR_OFF;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const unsigned long long lim = p.wait_limit_ns;
+
+  // this CTA's (b, h) and resident block; the streamed blocks it visits
+  const int bh = blockIdx.x / p.nblk;
+  const int blk = blockIdx.x - bh * p.nblk;
+  const int b = bh / p.H, h = bh - b * p.H;
+  // causal: key block j meets query blocks j .. nblk-1, query block i meets
+  // key blocks 0 .. i
+  const int first = (KV && p.causal) ? blk : 0;
+  const int last = (!KV && p.causal) ? blk : p.nblk - 1;
+  const int count = last - first + 1;
+
+  if (threadIdx.x == 0) {
+    // P / dS written: one arrival per compute warp; the rest are single
+    for (int i = 0; i < C::NUM_BARS; ++i) mbar_init(bars + 8 * i, i == C::B_PDS_FULL ? 4 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::PRODUCER_WARP && lane == 0) {
+    tma_prefetch_desc(&p.tmap_q);
+    tma_prefetch_desc(&p.tmap_k);
+    tma_prefetch_desc(&p.tmap_v);
+    tma_prefetch_desc(&p.tmap_do);
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == C::PRODUCER_WARP) {
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      // resident pair: K_j, V_j (dkdv) or Q_i, dO_i (dq)
+      mbar_arrive_expect_tx(bars + 8 * C::B_RES_FULL, 2 * C::TILE_BYTES);
+      load_tile<HD>(base + C::SA_OFF, KV ? &p.tmap_k : &p.tmap_q, bars + 8 * C::B_RES_FULL,
+                    blk * 128, h, b);
+      load_tile<HD>(base + C::SB_OFF, KV ? &p.tmap_v : &p.tmap_do, bars + 8 * C::B_RES_FULL,
+                    blk * 128, h, b);
+      for (int it = 0; it < count; ++it) {
+        if (it > 0 && !(ok = wait_phase(bars + 8 * C::B_STR_EMPTY, (it - 1) & 1, abort_flag, lim,
+                                        (kRoleProducer << 8) | kSiteKvEmpty)))
+          break;
+        const int row0 = (first + it) * 128;
+        mbar_arrive_expect_tx(bars + 8 * C::B_STR_FULL, 2 * C::TILE_BYTES);
+        load_tile<HD>(base + C::SC_OFF, KV ? &p.tmap_q : &p.tmap_k, bars + 8 * C::B_STR_FULL,
+                      row0, h, b);
+        load_tile<HD>(base + C::SD_OFF, KV ? &p.tmap_do : &p.tmap_v, bars + 8 * C::B_STR_FULL,
+                      row0, h, b);
+        ++issued;
+      }
+      if (!ok) {
+        // let the loads in flight land before the shared memory goes away
+        volatile int no_abort = 0;
+        wait_phase(bars + 8 * C::B_RES_FULL, 0, &no_abort, 10000000ull,
+                   (kRoleProducer << 8) | kSiteDrain);
+        if (issued > 0)
+          wait_phase(bars + 8 * C::B_STR_FULL, (issued - 1) & 1, &no_abort, 10000000ull,
+                     (kRoleProducer << 8) | kSiteDrain);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    if (lane == 0) {
+      const uint32_t idesc_sq = f16_idesc(BF16, 128, 128, false);  // S-shaped: N = 128 rows
+      const uint32_t idesc_acc = f16_idesc(BF16, 128, HD, true);   // accumulators: N = HD
+      bool ok = wait_phase(bars + 8 * C::B_RES_FULL, 0, abort_flag, lim,
+                           (kRoleMma << 8) | kSiteQFull);
+      tc_fence_after_sync();
+      // K-major [128 x HD] operands: resident A-side tiles and streamed B-side tiles
+      const uint32_t a0 = sw128_desc_lo(base + C::SA_OFF, 16), a1 = sw128_desc_lo(base + C::SB_OFF, 16);
+      const uint32_t b0 = sw128_desc_lo(base + C::SC_OFF, 16), b1 = sw128_desc_lo(base + C::SD_OFF, 16);
+      // 16-bit [128 x 128] tiles written by the compute warps (K-major, K = 128)
+      const uint32_t pt = sw128_desc_lo(base + C::SP_OFF, 16), dst = sw128_desc_lo(base + C::SDS_OFF, 16);
+      // MN-major B operands of the accumulating products: [K = 128 rows x N = HD]
+      // streamed tiles (Q for dK, K for dQ; dO for dV)
+      const uint32_t mq = sw128_desc_lo(base + C::SC_OFF, C::CHUNK_BYTES);
+      const uint32_t md = sw128_desc_lo(base + C::SD_OFF, C::CHUNK_BYTES);
+      for (int it = 0; ok && it < count; ++it) {
+        if (!(ok = wait_phase(bars + 8 * C::B_STR_FULL, it & 1, abort_flag, lim,
+                              (kRoleMma << 8) | kSiteKvFull)))
+          break;
+        tc_fence_after_sync();
+        // dkdv: S^T = K Q^T, dP^T = V dO^T;  dq: S = Q K^T, dP = dO V^T
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + C::S_COL, desc_from_lo(a0 + off), desc_from_lo(b0 + off), idesc_sq,
+                 kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + C::DP_COL, desc_from_lo(a1 + off), desc_from_lo(b1 + off), idesc_sq,
+                 kk > 0 ? 1u : 0u);
+        }
+        tc_commit(bars + 8 * C::B_SD_FULL);
+        if (!(ok = wait_phase(bars + 8 * C::B_PDS_FULL, it & 1, abort_flag, lim,
+                              (kRoleMma << 8) | kSitePFull)))
+          break;
+        tc_fence_after_sync();
+        // the 16-bit tiles contract over their 128 columns in 8 K-steps
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ka = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          const uint32_t kb = (kk * 16 * 128) >> 4;
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          if (KV) {
+            // dV += P^T dO, dK += dS^T Q
+            mma_ss(tmem + C::ACC0_COL, desc_from_lo(pt + ka), desc_from_lo(md + kb), idesc_acc, acc);
+            mma_ss(tmem + C::ACC1_COL, desc_from_lo(dst + ka), desc_from_lo(mq + kb), idesc_acc, acc);
+          } else {
+            // dQ += dS K
+            mma_ss(tmem + C::ACC0_COL, desc_from_lo(dst + ka), desc_from_lo(mq + kb), idesc_acc, acc);
+          }
+        }
+        // frees the streamed tiles and the 16-bit tiles
+        tc_commit(bars + 8 * C::B_STR_EMPTY);
+      }
+      if (ok) {
+        tc_commit(bars + 8 * C::B_DONE);
+      } else {
+        volatile int no_abort = 0;
+        tc_commit(bars + 8 * C::B_DRAIN);
+        wait_phase(bars + 8 * C::B_DRAIN, 0, &no_abort, 10000000ull, (kRoleMma << 8) | kSiteDrain);
+      }
+    }
+  } else {
+    // compute warps: thread = tile row = TMEM lane
+    const int r = warp * 32 + lane;
+    const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp) * 32u) << 16);
+    const float sl2 = p.scale_log2;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const long long vec0 = static_cast<long long>(bh) * p.N;
+    const int my_row = blk * 128 + r;  // key row (dkdv) or query row (dq)
+    float my_lse2 = INFINITY, my_dsum = 0.f;
+    if (!KV && my_row < p.N) {
+      my_lse2 = p.lse[vec0 + my_row] * kLog2e;
+      my_dsum = p.dsum[vec0 + my_row];
+    }
+    bool ok = true;
+    for (int it = 0; it < count; ++it) {
+      const int other0 = (first + it) * 128;  // first streamed row of this step
+      if (KV) {
+        // per-column statistics of the streamed query block (+inf lse masks
+        // query rows past N)
+        __syncwarp();
+#pragma unroll
+        for (int c = lane; c < 128; c += 32) {
+          const int qi = other0 + c;
+          lse2_s[c] = qi < p.N ? p.lse[vec0 + qi] * kLog2e : INFINITY;
+          dsum_s[c] = qi < p.N ? p.dsum[vec0 + qi] : 0.f;
+        }
+        __syncwarp();
+      }
+      ok = wait_phase(bars + 8 * C::B_SD_FULL, it & 1, abort_flag, lim,
+                      (kRoleSoftmax << 8) | kSiteSFull);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after_sync();
+      // the 16-bit tiles of the previous step have been read
+      if (it > 0) {
+        ok = wait_phase(bars + 8 * C::B_STR_EMPTY, (it - 1) & 1, abort_flag, lim,
+                        (kRoleSoftmax << 8) | kSitePFree);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after_sync();
+      }
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32_sync(lane_base + C::S_COL + c0, sv);
+        tmem_ld32_sync(lane_base + C::DP_COL + c0, dv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float pp[2], ds[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = c0 + 2 * q + e;
+            const float s = __uint_as_float(sv[2 * q + e]);
+            const float dpv = __uint_as_float(dv[2 * q + e]);
+            float pv;
+            if (KV) {
+              // row = key my_row, column = query other0 + c
+              const bool vis = !p.causal || other0 + c >= my_row;
+              pv = vis ? ex2(s * sl2 - lse2_s[c]) : 0.f;
+              ds[e] = pv * (dpv - dsum_s[c]);
+            } else {
+              // row = query my_row, column = key other0 + c
+              const int key = other0 + c;
+              const bool vis = key < p.N && (!p.causal || key <= my_row);
+              pv = vis ? ex2(s * sl2 - my_lse2) : 0.f;
+              ds[e] = pv * (dpv - my_dsum);
+            }
+            pp[e] = pv;
+          }
+          pk[q] = pack2<BF16>(pp[0], pp[1]);
+          dk[q] = pack2<BF16>(ds[0], ds[1]);
+        }
+        if (KV) store_row32(base + C::SP_OFF, r, c0, pk);
+        store_row32(base + C::SDS_OFF, r, c0, dk);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * C::B_PDS_FULL);
+    }
+    if (ok) {
+      ok = wait_phase(bars + 8 * C::B_DONE, 0, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after_sync();
+        using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+        const long long row_off = (vec0 + my_row) * HD;
+#pragma unroll 1
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t a0[32], a1[32];
+          tmem_ld32_sync(lane_base + C::ACC0_COL + c, a0);
+          if (KV) tmem_ld32_sync(lane_base + C::ACC1_COL + c, a1);
+          if (my_row < p.N) {
+            if (KV) {
+              store_acc32<BF16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f);
+              store_acc32<BF16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale);
+            } else {
+              store_acc32<BF16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    __syncwarp();
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa_sm100

@@ -90,6 +90,33 @@ int fa_fwd_qkvpacked(const void *qkv, void *o, float *lse, int B, int N, int H, 
                      int causal, float dropout_p, int dtype, struct CUstream_st *stream);
 
 /* Static text for a status code. */
+/*
+ * Gradient of fa_fwd: dQ, dK, dV for an upstream gradient dO of O.  The score
+ * tile is recomputed from q, k and the forward's logsumexp, the
+ * recomputation in the backward pass that sections 1 and 7 of the
+ * intelliparadigm.com build guide describe; the rest is the chain rule through
+ * the forward (dV = P^T dO, dS = P * (dO V^T - rowsum(dO * O)),
+ * dQ = scale dS K, dK = scale dS^T Q).
+ *
+ *   q, k, v, o : [B, H, N, d] contiguous, element type `dtype` (read only);
+ *                o and lse are the outputs of fa_fwd on the same q, k, v,
+ *                scale and causal
+ *   lse        : [B, H, N] fp32 (read only; required)
+ *   dout       : [B, H, N, d] contiguous, element type `dtype` (read only)
+ *   dq, dk, dv : [B, H, N, d] contiguous, element type `dtype` (written)
+ *   workspace  : [B, H, N] fp32, caller-owned scratch (overwritten); the
+ *                library allocates nothing
+ *   d          : 64 or 128 (else FA_ERR_HEADDIM)
+ *   scale, causal, dtype, stream: as fa_fwd
+ *
+ * Asynchronous on `stream`: three kernels (row statistic, dK/dV, dQ).
+ * Returns FA_OK or a negative status; FA_ERR_ALIGN if a tensor pointer is not
+ * 16-byte aligned or lse / workspace not 4-byte aligned.
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dout, void *dq, void *dk, void *dv, float *workspace, int B, int H, int N,
+           int d, float scale, int causal, int dtype, struct CUstream_st *stream);
+
 const char *fa_strerror(int status);
 
 /*

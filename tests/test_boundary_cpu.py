@@ -109,3 +109,20 @@ def test_library_has_no_torch_dependency():
 def test_exp2_hook_argument_check(lib):
     assert lib.fa_debug_exp2_poly(None, P, 4, None) == fa.FA_ERR_ARG
     assert lib.fa_debug_exp2_poly(P, P, -1, None) == fa.FA_ERR_ARG
+
+
+def test_bwd_argument_errors(lib):
+    def call(q=P, o=P, lse=P, ws=P, B=1, H=1, N=128, d=128, scale=0.0, causal=0, dtype=1):
+        return lib.fa_bwd(q, P, P, o, lse, P, P, P, P, ws, B, H, N, d, scale, causal, dtype, None)
+    assert call(q=None) == fa.FA_ERR_ARG
+    assert call(lse=None) == fa.FA_ERR_ARG
+    assert call(ws=None) == fa.FA_ERR_ARG
+    assert call(N=0) == fa.FA_ERR_ARG
+    assert call(d=256) == fa.FA_ERR_HEADDIM
+    assert call(d=96) == fa.FA_ERR_HEADDIM
+    assert call(dtype=3) == fa.FA_ERR_DTYPE
+    assert call(scale=float("nan")) == fa.FA_ERR_ARG
+    assert call(q=P + 8) == fa.FA_ERR_ALIGN
+    assert call(o=P + 2) == fa.FA_ERR_ALIGN
+    assert call(lse=P + 2) == fa.FA_ERR_ALIGN
+    assert call(ws=P + 1) == fa.FA_ERR_ALIGN
