@@ -24,6 +24,12 @@ constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
 constexpr unsigned long long kWaitLimitNs = FA_WAIT_LIMIT_NS;
 constexpr int kMaxDevices = 64;
 
+// Row-statistic scratch of fa_bwd_noalloc: a library-owned device array, one
+// per device (each device's module instance has its own), so that entry point
+// needs no caller workspace and allocates nothing.
+constexpr long long kBwdScratchFloats = 1ll << 23;
+static __device__ __align__(256) float g_bwd_scratch[kBwdScratchFloats];
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -37,6 +43,7 @@ struct DeviceState {
   int sm_count = 0;
   bool attr_set[6] = {false, false, false, false, false, false};
   bool bwd_attr_set[8] = {false, false, false, false, false, false, false, false};
+  float* bwd_scratch = nullptr;  // this device's g_bwd_scratch
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -238,26 +245,49 @@ int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int N, int H, 
              sb, hd, d, (long long)N * hd, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-           const void* dout, void* dq, void* dk, void* dv, float* workspace, int B, int H, int N,
-           int d, float scale, int causal, int dtype, struct CUstream_st* stream) {
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_ARG;
-  int rc = check_common(B, H, N, d, &scale, causal, dtype);
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by both backward entry points (workspace checked by
+// the caller of this function when it has one).
+int check_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+              const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+              float* scale, int causal, int dtype) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_ARG;
+  int rc = check_common(B, H, N, d, scale, causal, dtype);
   if (rc != FA_OK) return rc;
   if (d != 64 && d != 128) return FA_ERR_HEADDIM;
   for (const void* t : {q, k, v, o, dout, static_cast<const void*>(dq), static_cast<const void*>(dk),
                         static_cast<const void*>(dv)})
     if (!aligned16(t)) return FA_ERR_ALIGN;
-  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || (reinterpret_cast<uintptr_t>(workspace) & 3u) != 0)
-    return FA_ERR_ALIGN;
-  const int nblk = (N + 127) / 128;
-  if ((long long)B * H * nblk > 0x7fffffffLL) return FA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return FA_ERR_ALIGN;
+  if ((long long)B * H * ((N + 127) / 128) > 0x7fffffffLL) return FA_ERR_ARG;
+  return FA_OK;
+}
 
+// Encodes the operands and launches the three backward kernels.  A null
+// `workspace` selects this device's library-owned scratch array.
+int run_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+            const void* dout, void* dq, void* dk, void* dv, float* workspace, int B, int H, int N,
+            int d, float scale, int causal, int dtype, cudaStream_t s) {
   std::lock_guard<std::mutex> lock(g_mutex);
-  if ((rc = get_encode_fn()) != FA_OK) return rc;
+  int rc = get_encode_fn();
+  if (rc != FA_OK) return rc;
   DeviceState* st = nullptr;
   int dev = 0;
   if ((rc = device_state(&st, &dev)) != FA_OK) return rc;
+  if (workspace == nullptr) {
+    if (st->bwd_scratch == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+      }
+      st->bwd_scratch = static_cast<float*>(ptr);
+    }
+    workspace = st->bwd_scratch;
+  }
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const long long sn = d, sh = (long long)N * d, sb = (long long)H * N * d;
@@ -278,12 +308,36 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   p.causal = causal;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.nblk = nblk;
+  p.nblk = (N + 127) / 128;
   p.wait_limit_ns = kWaitLimitNs;
   const bool bf16 = dtype == FA_BF16;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) return bf16 ? launch_bwd<64, true>(p, *st, s) : launch_bwd<64, false>(p, *st, s);
   return bf16 ? launch_bwd<128, true>(p, *st, s) : launch_bwd<128, false>(p, *st, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dout, void* dq, void* dk, void* dv, float* workspace, int B, int H, int N,
+           int d, float scale, int causal, int dtype, struct CUstream_st* stream) {
+  int rc = check_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, &scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (!workspace) return FA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 3u) != 0) return FA_ERR_ALIGN;
+  return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, H, N, d, scale, causal, dtype,
+                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                   float scale, int causal, int dtype, struct CUstream_st* stream) {
+  int rc = check_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, &scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if ((long long)B * H * N > kBwdScratchFloats) return FA_ERR_ARG;
+  return run_bwd(q, k, v, o, lse, dout, dq, dk, dv, nullptr, B, H, N, d, scale, causal, dtype,
+                 reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* fa_strerror(int status) {

@@ -31,6 +31,8 @@ SIGNATURES = {
     "fa_fwd_qkvpacked": (_I, [_VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I,
                     _VP]),
+    "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I,
+                            _I, _VP]),
     "fa_strerror": (ctypes.c_char_p, [_I]),
     "fa_device_status": (_I, [_I, ctypes.POINTER(ctypes.c_uint)]),
     "fa_debug_watchdog_selftest": (_I, [ctypes.c_ulonglong, _VP]),
@@ -181,6 +183,30 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
                        _DT[q.dtype], _stream_ptr(q))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                lse: torch.Tensor, dout: torch.Tensor, scale: float | None = None,
+                causal: bool = False):
+    """:func:`bwd` through ``fa_bwd_noalloc``: the row statistic lives in the
+    library's own device array instead of a workspace tensor."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_tensor(t, name)
+    if not (q.shape == k.shape == v.shape == o.shape == dout.shape) or q.dim() != 4:
+        raise ValueError("q, k, v, o, dout must share one [B, H, N, d] shape")
+    if len({t.dtype for t in (q, k, v, o, dout)}) != 1:
+        raise ValueError("q, k, v, o, dout must share one dtype")
+    B, H, N, d = q.shape
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous [B, H, N] float32 tensor")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                               lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), B, H, N, d, 0.0 if scale is None else float(scale),
+                               int(bool(causal)), _DT[q.dtype], _stream_ptr(q))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -117,6 +117,21 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            const void *dout, void *dq, void *dk, void *dv, float *workspace, int B, int H, int N,
            int d, float scale, int causal, int dtype, struct CUstream_st *stream);
 
+/*
+ * fa_bwd without the workspace argument: the fp32 row statistic goes into a
+ * device array the library owns (a file-scope __device__ array, one per
+ * device), so the call allocates nothing and the caller provides no scratch.
+ *
+ *   B * H * N must not exceed 8,388,608 (the array's size), else FA_ERR_ARG.
+ *   The array is shared by every call on the device: two calls that may run
+ *   at the same time (on different streams) must not both use this entry
+ *   point; calls ordered on one stream may.
+ *   Other arguments, results and errors as fa_bwd.
+ */
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                   const void *dout, void *dq, void *dk, void *dv, int B, int H, int N, int d,
+                   float scale, int causal, int dtype, struct CUstream_st *stream);
+
 const char *fa_strerror(int status);
 
 /*
