@@ -187,7 +187,7 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
 
 template <int HD, bool BF16, bool KV>
 int launch_bwd_kernel(const BwdParams& p, DeviceState& st, cudaStream_t stream) {
-  using C = BwdCfg<HD>;
+  using C = BwdCfg<HD, KV>;
   auto kernel = fa_bwd_kernel<HD, BF16, KV>;
   const int slot = (HD == 64 ? 0 : 4) + (BF16 ? 2 : 0) + (KV ? 1 : 0);
   if (!st.bwd_attr_set[slot]) {

@@ -50,7 +50,7 @@ struct BwdParams {
   unsigned long long wait_limit_ns;
 };
 
-template <int HD>
+template <int HD, bool KV>
 struct BwdCfg {
   static_assert(HD == 64 || HD == 128, "backward head dim");
   static constexpr int CHUNKS = HD / 64;
@@ -59,19 +59,28 @@ struct BwdCfg {
   static constexpr int SQR_BYTES = 2 * CHUNK_BYTES;         // one [128 x 128] 16-bit tile
   static constexpr int THREADS = 192;
   static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
-  // shared memory: the two resident tiles, the two streamed tiles, the 16-bit
-  // P^T / dS^T tiles (dkdv) or dS tile (dq), two 128-float vectors, barriers
+  // Shared memory: the resident pair (K, V for dK/dV; Q, dO for dQ), STAGES
+  // slots of the streamed pair (Q, dO / K, V), the 16-bit P^T and dS^T tiles
+  // (dK/dV) or dS tile (dQ), per-warp column statistics (dK/dV), barriers.
+  // Two streamed slots where they fit, so the next block loads while this one
+  // is computed.
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int SQR_TILES = KV ? 2 : 1;
+  static constexpr int VEC_BYTES = KV ? 4 * 2 * 128 * 4 : 0;
+  static constexpr int B_RES_FULL = 0, B_STR_FULL = 1 /* [stage] */, B_STR_EMPTY = 3 /* [stage] */,
+                       B_SD_FULL = 5, B_PDS_FULL = 6, B_PDS_FREE = 7, B_DONE = 8, B_DRAIN = 9,
+                       NUM_BARS = 10;
+  static constexpr int FIXED_BYTES = 2 * TILE_BYTES + SQR_TILES * SQR_BYTES + VEC_BYTES +
+                                     NUM_BARS * 8 + 16 + 1024;
+  static constexpr int STAGES = FIXED_BYTES + 2 * STAGE_BYTES <= 232448 ? 2 : 1;
   static constexpr int SA_OFF = 0;                           // K (dkdv) / Q (dq)
   static constexpr int SB_OFF = TILE_BYTES;                  // V (dkdv) / dO (dq)
-  static constexpr int SC_OFF = 2 * TILE_BYTES;              // Q (dkdv) / K (dq)
-  static constexpr int SD_OFF = 3 * TILE_BYTES;              // dO (dkdv) / V (dq)
-  static constexpr int SP_OFF = 4 * TILE_BYTES;              // P^T (dkdv)
-  static constexpr int SDS_OFF = SP_OFF + SQR_BYTES;         // dS^T (dkdv) / dS (dq)
-  // per compute warp: lse*log2e [128] and D [128] of the streamed query block
+  static constexpr int SSTR_OFF = 2 * TILE_BYTES;            // slot s: Q / K at +s*STAGE_BYTES,
+                                                             // dO / V at +TILE_BYTES
+  static constexpr int SP_OFF = SSTR_OFF + STAGES * STAGE_BYTES;  // P^T (dkdv only)
+  static constexpr int SDS_OFF = SP_OFF + (KV ? SQR_BYTES : 0);   // dS^T (dkdv) / dS (dq)
   static constexpr int VEC_OFF = SDS_OFF + SQR_BYTES;
-  static constexpr int BAR_OFF = VEC_OFF + 4 * 2 * 128 * 4;
-  static constexpr int B_RES_FULL = 0, B_STR_FULL = 1, B_STR_EMPTY = 2, B_SD_FULL = 3,
-                       B_PDS_FULL = 4, B_DONE = 5, B_DRAIN = 6, NUM_BARS = 7;
+  static constexpr int BAR_OFF = VEC_OFF + VEC_BYTES;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int END_OFF = MISC_OFF + 16;
   static constexpr int SMEM_BYTES = END_OFF + 1024;  // + slack to align the base to 1024
@@ -139,9 +148,9 @@ __device__ __forceinline__ void store_acc32(void* dst_row, const uint32_t* acc, 
 // KV = true: the dK/dV kernel (CTA per key block, streams Q and dO).
 // KV = false: the dQ kernel (CTA per query block, streams K and V).
 template <int HD, bool BF16, bool KV>
-__global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
+__global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ BwdParams p) {
-  using C = BwdCfg<HD>;
+  using C = BwdCfg<HD, KV>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -198,15 +207,16 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       load_tile<HD>(base + C::SB_OFF, KV ? &p.tmap_v : &p.tmap_do, bars + 8 * C::B_RES_FULL,
                     blk * 128, h, b);
       for (int it = 0; it < count; ++it) {
-        if (it > 0 && !(ok = wait_phase(bars + 8 * C::B_STR_EMPTY, (it - 1) & 1, abort_flag, lim,
-                                        (kRoleProducer << 8) | kSiteKvEmpty)))
+        const int stage = it % C::STAGES, use = it / C::STAGES;
+        if (use > 0 && !(ok = wait_phase(bars + 8 * (C::B_STR_EMPTY + stage), (use - 1) & 1,
+                                         abort_flag, lim, (kRoleProducer << 8) | kSiteKvEmpty)))
           break;
         const int row0 = (first + it) * 128;
-        mbar_arrive_expect_tx(bars + 8 * C::B_STR_FULL, 2 * C::TILE_BYTES);
-        load_tile<HD>(base + C::SC_OFF, KV ? &p.tmap_q : &p.tmap_k, bars + 8 * C::B_STR_FULL,
-                      row0, h, b);
-        load_tile<HD>(base + C::SD_OFF, KV ? &p.tmap_do : &p.tmap_v, bars + 8 * C::B_STR_FULL,
-                      row0, h, b);
+        const uint32_t full = bars + 8 * (C::B_STR_FULL + stage);
+        const uint32_t slot = base + C::SSTR_OFF + stage * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(full, 2 * C::TILE_BYTES);
+        load_tile<HD>(slot, KV ? &p.tmap_q : &p.tmap_k, full, row0, h, b);
+        load_tile<HD>(slot + C::TILE_BYTES, KV ? &p.tmap_do : &p.tmap_v, full, row0, h, b);
         ++issued;
       }
       if (!ok) {
@@ -214,9 +224,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
         volatile int no_abort = 0;
         wait_phase(bars + 8 * C::B_RES_FULL, 0, &no_abort, 10000000ull,
                    (kRoleProducer << 8) | kSiteDrain);
-        if (issued > 0)
-          wait_phase(bars + 8 * C::B_STR_FULL, (issued - 1) & 1, &no_abort, 10000000ull,
-                     (kRoleProducer << 8) | kSiteDrain);
+        for (int k = issued > C::STAGES ? issued - C::STAGES : 0; k < issued; ++k)
+          wait_phase(bars + 8 * (C::B_STR_FULL + k % C::STAGES), (k / C::STAGES) & 1, &no_abort,
+                     10000000ull, (kRoleProducer << 8) | kSiteDrain);
       }
     }
   } else if (warp == C::MMA_WARP) {
@@ -228,16 +238,19 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       tc_fence_after_sync();
       // K-major [128 x HD] operands: resident A-side tiles and streamed B-side tiles
       const uint32_t a0 = sw128_desc_lo(base + C::SA_OFF, 16), a1 = sw128_desc_lo(base + C::SB_OFF, 16);
-      const uint32_t b0 = sw128_desc_lo(base + C::SC_OFF, 16), b1 = sw128_desc_lo(base + C::SD_OFF, 16);
       // 16-bit [128 x 128] tiles written by the compute warps (K-major, K = 128)
       const uint32_t pt = sw128_desc_lo(base + C::SP_OFF, 16), dst = sw128_desc_lo(base + C::SDS_OFF, 16);
-      // MN-major B operands of the accumulating products: [K = 128 rows x N = HD]
-      // streamed tiles (Q for dK, K for dQ; dO for dV)
-      const uint32_t mq = sw128_desc_lo(base + C::SC_OFF, C::CHUNK_BYTES);
-      const uint32_t md = sw128_desc_lo(base + C::SD_OFF, C::CHUNK_BYTES);
       for (int it = 0; ok && it < count; ++it) {
-        if (!(ok = wait_phase(bars + 8 * C::B_STR_FULL, it & 1, abort_flag, lim,
-                              (kRoleMma << 8) | kSiteKvFull)))
+        const int stage = it % C::STAGES;
+        const uint32_t slot = base + C::SSTR_OFF + stage * C::STAGE_BYTES;
+        // the streamed pair as K-major B of S / dP ...
+        const uint32_t b0 = sw128_desc_lo(slot, 16), b1 = sw128_desc_lo(slot + C::TILE_BYTES, 16);
+        // ... and as MN-major B [K = 128 rows x N = HD] of the accumulating
+        // products (Q for dK, K for dQ; dO for dV)
+        const uint32_t mq = sw128_desc_lo(slot, C::CHUNK_BYTES);
+        const uint32_t md = sw128_desc_lo(slot + C::TILE_BYTES, C::CHUNK_BYTES);
+        if (!(ok = wait_phase(bars + 8 * (C::B_STR_FULL + stage), (it / C::STAGES) & 1, abort_flag,
+                              lim, (kRoleMma << 8) | kSiteKvFull)))
           break;
         tc_fence_after_sync();
         // dkdv: S^T = K Q^T, dP^T = V dO^T;  dq: S = Q K^T, dP = dO V^T
@@ -273,8 +286,9 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
             mma_ss(tmem + C::ACC0_COL, desc_from_lo(dst + ka), desc_from_lo(mq + kb), idesc_acc, acc);
           }
         }
-        // frees the streamed tiles and the 16-bit tiles
-        tc_commit(bars + 8 * C::B_STR_EMPTY);
+        // frees the streamed slot and the 16-bit tiles
+        tc_commit(bars + 8 * (C::B_STR_EMPTY + stage));
+        tc_commit(bars + 8 * C::B_PDS_FREE);
       }
       if (ok) {
         tc_commit(bars + 8 * C::B_DONE);
@@ -318,7 +332,7 @@ __global__ void __launch_bounds__(BwdCfg<HD>::THREADS, 1)
       tc_fence_after_sync();
       // the 16-bit tiles of the previous step have been read
       if (it > 0) {
-        ok = wait_phase(bars + 8 * C::B_STR_EMPTY, (it - 1) & 1, abort_flag, lim,
+        ok = wait_phase(bars + 8 * C::B_PDS_FREE, (it - 1) & 1, abort_flag, lim,
                         (kRoleSoftmax << 8) | kSitePFree);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after_sync();
