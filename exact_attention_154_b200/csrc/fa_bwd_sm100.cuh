@@ -21,10 +21,11 @@
 // bwd_dq_kernel: one CTA per 128-query block i; recomputes S and dP the same
 // way for every key block j and accumulates dQ_i += dS K_j in TMEM.
 //
-// Roles per CTA (192 threads): warps 0-3 compute P and dS (thread = TMEM
-// lane = tile row), warp 4 streams tiles with TMA, warp 5 owns TMEM and one of
-// its threads issues every tcgen05.mma.  Q/dO (resp. K/V) of the streamed
-// operand are single-buffered.  All mbarrier waits are bounded (wait_phase).
+// Roles per CTA (320 threads): warps 0-7 compute P and dS (thread = TMEM
+// lane = tile row; warps 0-3 take columns 0-63 of each block, warps 4-7
+// columns 64-127), warp 8 streams tiles with TMA, warp 9 owns TMEM and one of
+// its threads issues every tcgen05.mma.  The streamed pair has two slots
+// where shared memory allows.  All mbarrier waits are bounded (wait_phase).
 #pragma once
 
 #include "fa_fwd_sm100.cuh"
@@ -57,8 +58,11 @@ struct BwdCfg {
   static constexpr int CHUNK_BYTES = 128 * 128;
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;   // one [128 x HD] 16-bit tile
   static constexpr int SQR_BYTES = 2 * CHUNK_BYTES;         // one [128 x 128] 16-bit tile
-  static constexpr int THREADS = 192;
-  static constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
+  // two compute warpgroups (key/query rows x 64 of the 128 columns each),
+  // then the producer warp and the MMA warp
+  static constexpr int COMPUTE_WARPS = 8;
+  static constexpr int THREADS = 32 * (COMPUTE_WARPS + 2);
+  static constexpr int PRODUCER_WARP = COMPUTE_WARPS, MMA_WARP = COMPUTE_WARPS + 1;
   // Shared memory: the resident pair (K, V for dK/dV; Q, dO for dQ), STAGES
   // slots of the streamed pair (Q, dO / K, V), the 16-bit P^T and dS^T tiles
   // (dK/dV) or dS tile (dQ), per-warp column statistics (dK/dV), barriers.
@@ -66,7 +70,7 @@ struct BwdCfg {
   // is computed.
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int SQR_TILES = KV ? 2 : 1;
-  static constexpr int VEC_BYTES = KV ? 4 * 2 * 128 * 4 : 0;
+  static constexpr int VEC_BYTES = KV ? COMPUTE_WARPS * 2 * 64 * 4 : 0;
   static constexpr int B_RES_FULL = 0, B_STR_FULL = 1 /* [stage] */, B_STR_EMPTY = 3 /* [stage] */,
                        B_SD_FULL = 5, B_PDS_FULL = 6, B_PDS_FREE = 7, B_DONE = 8, B_DRAIN = 9,
                        NUM_BARS = 10;
@@ -157,10 +161,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   uint8_t* smem = smem_raw + (base - raw);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-  // this warp's copy of the per-column statistics (no cross-warp barrier, so
-  // a warp that leaves on an abandoned wait cannot strand the others)
-  float* lse2_s = reinterpret_cast<float*>(smem + C::VEC_OFF) + (threadIdx.x / 32 % 4) * 256;
-  float* dsum_s = lse2_s + 128;
+  // this warp's copy of the statistics of its 64 columns (no cross-warp
+  // barrier, so a warp that leaves on an abandoned wait cannot strand the others)
+  float* lse2_s = reinterpret_cast<float*>(smem + C::VEC_OFF) + (threadIdx.x / 32) * 128;
+  float* dsum_s = lse2_s + 64;
   const uint32_t bars = base + C::BAR_OFF;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const unsigned long long lim = p.wait_limit_ns;
@@ -177,7 +181,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     // P / dS written: one arrival per compute warp; the rest are single
-    for (int i = 0; i < C::NUM_BARS; ++i) mbar_init(bars + 8 * i, i == C::B_PDS_FULL ? 4 : 1);
+    for (int i = 0; i < C::NUM_BARS; ++i)
+      mbar_init(bars + 8 * i, i == C::B_PDS_FULL ? C::COMPUTE_WARPS : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -299,9 +304,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       }
     }
   } else {
-    // compute warps: thread = tile row = TMEM lane
-    const int r = warp * 32 + lane;
-    const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp) * 32u) << 16);
+    // compute warps: thread = tile row = TMEM lane; this warpgroup's 64 columns
+    const int quad = warp % 4, cb = 64 * (warp / 4);
+    const int r = quad * 32 + lane;
+    const uint32_t lane_base = tmem + ((static_cast<uint32_t>(quad) * 32u) << 16);
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     const long long vec0 = static_cast<long long>(bh) * p.N;
@@ -319,8 +325,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         // query rows past N)
         __syncwarp();
 #pragma unroll
-        for (int c = lane; c < 128; c += 32) {
-          const int qi = other0 + c;
+        for (int c = lane; c < 64; c += 32) {
+          const int qi = other0 + cb + c;
           lse2_s[c] = qi < p.N ? p.lse[vec0 + qi] * kLog2e : INFINITY;
           dsum_s[c] = qi < p.N ? p.dsum[vec0 + qi] : 0.f;
         }
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         tc_fence_after_sync();
       }
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = cb; c0 < cb + 64; c0 += 32) {
         uint32_t sv[32], dv[32];
         tmem_ld32_sync(lane_base + C::S_COL + c0, sv);
         tmem_ld32_sync(lane_base + C::DP_COL + c0, dv);
@@ -355,8 +361,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
             if (KV) {
               // row = key my_row, column = query other0 + c
               const bool vis = !p.causal || other0 + c >= my_row;
-              pv = vis ? ex2(s * sl2 - lse2_s[c]) : 0.f;
-              ds[e] = pv * (dpv - dsum_s[c]);
+              pv = vis ? ex2(s * sl2 - lse2_s[c - cb]) : 0.f;
+              ds[e] = pv * (dpv - dsum_s[c - cb]);
             } else {
               // row = query my_row, column = key other0 + c
               const int key = other0 + c;
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
         const long long row_off = (vec0 + my_row) * HD;
 #pragma unroll 1
-        for (int c = 0; c < HD; c += 32) {
+        for (int c = (warp / 4) * (HD / 2); c < (warp / 4 + 1) * (HD / 2); c += 32) {
           uint32_t a0[32], a1[32];
           tmem_ld32_sync(lane_base + C::ACC0_COL + c, a0);
           if (KV) tmem_ld32_sync(lane_base + C::ACC1_COL + c, a1);
