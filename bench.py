@@ -43,6 +43,7 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fa_fwd_sm100_traffic.md")
 KERNEL_SOURCES = ["exact_attention_154_b200/csrc/fa_fwd_sm100.cuh",
+                  "exact_attention_154_b200/csrc/fa_bwd_sm100.cuh",
                   "exact_attention_154_b200/csrc/sm100_ptx.cuh",
                   "exact_attention_154_b200/csrc/fa_api.cu"]
 
@@ -447,7 +448,8 @@ def bench_gpu_bwd(args, w, key, world, rank, local):
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "peak_note": f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json)"
                                   if peak_src == "measured" else "fallback 1.59 PFLOP/s",
-                     "traffic": None,
+                     # DRAM bytes of all three kernels of one step (ncu)
+                     "traffic": profiled_traffic("bwd:" + key),
                      "algorithmic_bytes": 8 * nd * e + 12 * w.B * w.H * w.N,
                      "kernel": "fa_bwd_kernel", "launches_per_step": 3},
         "e2e": {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
