@@ -12,21 +12,24 @@
 //     (b, h, 256 query rows = two 128-row Q tiles, or one for head dim 256);
 //   * a TMA producer warp loads the Q tiles once per work tile and streams
 //     128-row K and V tiles through a ring of shared-memory stages guarded by
-//     full / empty mbarriers (128-byte swizzle, no cluster multicast), K one
-//     block ahead of V;
-//   * one thread of the MMA warp issues tcgen05 MMAs: S = Q K^T into tensor
-//     memory (TMEM) and O += P V, both from shared-memory operands, committing
-//     each group to an mbarrier;
+//     full / empty mbarriers (128-byte swizzle; every CTA loads its own
+//     tiles), K one block ahead of V;
+//   * two threads issue the tcgen05 MMAs, one per product, because a thread
+//     that issues MMAs runs only about one instruction ahead of the tensor
+//     pipe: one issues S = Q K^T into tensor memory (TMEM), the other
+//     O += P V with P from shared memory, each committing its groups to
+//     mbarriers;
 //   * two softmax warpgroups own each Q tile, one per 64 key columns: thread t
 //     of a group owns query row t (TMEM lane t), so the row max and row sum
 //     need no shuffles, only one exchange per block between the two groups
 //     through shared memory.  Each group reads its half of S from TMEM and,
 //     once the row max is agreed, releases the S buffer so the tensor core can
 //     already compute the next block's S; then it applies scale (in the log2
-//     domain), the causal / ragged mask and the online update, writes its
-//     half of P as 16-bit values into shared memory in the layout the MMA
-//     reads, rescales its half of O in TMEM when the reference max moved, and
-//     finally writes its half of O / l and (one group) the logsumexp.
+//     domain), the causal / ragged mask and the online update, rescales its
+//     half of O in TMEM when the reference max moved, writes its half of P as
+//     16-bit values into the one shared-memory P tile the Q tiles use in turn
+//     (handed over by 64-key halves), and finally writes its half of O / l
+//     and (one group) the logsumexp.
 //
 // Because S(j+1) is computed while the softmax of block j runs, the softmax
 // groups work back to back; four of them share each SM sub-partition, which

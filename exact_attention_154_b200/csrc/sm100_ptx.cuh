@@ -4,7 +4,8 @@
 // plus the shared-memory and instruction descriptors those MMAs read.
 //
 // Everything here follows the public PTX ISA (tcgen05, cp.async.bulk.tensor,
-// mbarrier sections).  No TMA load here uses .multicast::cluster.
+// mbarrier sections).  Every TMA load here writes only the issuing CTA's own
+// shared memory; none is a cluster-wide load.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
