@@ -621,8 +621,8 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       x_mine[r] = m_half;
       if (!group_meet()) return;
       const float m_blk = fmaxf(m_half, x_other[r]);
-      // S is in registers and both groups have read the exchange slot: the MMA
-      // warp may overwrite the S buffer with S(j+1), and the slots are free
+      // S is in registers and both groups have read the exchange slot: the S
+      // thread may overwrite the S buffer with S(j+1), and the slots are free
       // again once that S arrives.
       tc_fence_before_sync();
       __syncwarp();
