@@ -16,7 +16,7 @@ namespace {
 
 using namespace fa_sm100;
 
-constexpr int kVersion = 1 * 10000 + 0 * 100 + 0;
+constexpr int kVersion = 1 * 10000 + 1 * 100 + 0;  // 1.1.0: the backward entry points
 // Limit of every mbarrier wait of the kernel (2 s unless the build sets it).
 #ifndef FA_WAIT_LIMIT_NS
 #define FA_WAIT_LIMIT_NS 2000000000ull

@@ -1,6 +1,7 @@
 /*
- * fa.h -- C ABI of the B200 (sm_100a) exact attention forward library
- * (libfa_sm100.so).
+ * fa.h -- C ABI of the B200 (sm_100a) exact attention library (libfa_sm100.so):
+ * the forward (fa_fwd, fa_fwd_qkvpacked) and its gradient (fa_bwd,
+ * fa_bwd_noalloc).
  *
  * Operation.  For every batch b, head h and query row i:
  *
@@ -22,7 +23,8 @@
  * before the P V product (as on the tensor cores of every FlashAttention).
  *
  * Memory.  Every pointer is device memory owned by the caller; the library
- * allocates nothing per call.  q, k, v, qkv and o must be 16-byte aligned.
+ * allocates nothing per call (fa_bwd_noalloc writes its row statistic into a
+ * device array the library owns).  Tensor pointers must be 16-byte aligned.
  *
  * Execution.  Calls are asynchronous on `stream` (a cudaStream_t; NULL is the
  * legacy default stream) and never synchronise.  The returned status covers
@@ -152,7 +154,7 @@ int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st *
 
 /*
  * Test hook: y[i] = the kernel's software 2^x (the FMA-pipe exponential used
- * for part of the softmax weights) for n device floats x.  Not part of the
+ * for a quarter of the softmax weights at head dim 256) for n device floats x.  Not part of the
  * attention method; exposed so that its error against exp2f can be measured.
  */
 int fa_debug_exp2_poly(const float *x, float *y, int n, struct CUstream_st *stream);
