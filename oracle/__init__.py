@@ -17,13 +17,17 @@ Three independent implementations live here:
   extended with the causal mask and the logsumexp output.
 * :func:`oracle.brute.attention_fsum` -- a scalar pure-Python version using
   ``math.fsum`` for tiny inputs.
+* :func:`attention_masked` -- the definition with a local window and an
+  ALiBi bias (the two masks the packed call names), pinned in
+  ``tests/test_oracle_mask_pins.py``.
 * :func:`attention_bwd` -- the gradient of the plain definition with respect
   to q, k, v (chain rule written out in ``fa_oracle.c``), pinned in
   ``tests/test_oracle_bwd_pins.py`` by central finite differences of
   :func:`attention`, closed forms and invariants.
 
 Parity status: every function here is pinned by tests in
-``tests/test_oracle_pins.py`` and ``tests/test_oracle_bwd_pins.py`` (closed
+``tests/test_oracle_pins.py``, ``tests/test_oracle_mask_pins.py`` and
+``tests/test_oracle_bwd_pins.py`` (closed
 forms, invariants, brute force, finite differences and the
 recurrence-equals-definition check); none is "parity unpinned".
 """
@@ -75,6 +79,11 @@ def _load():
                 dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
                 ctypes.c_int, dp]
             lib.oracle_attention_probs.restype = ctypes.c_int
+            lib.oracle_attention_fwd_masked.argtypes = [
+                dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                dp, ip, ctypes.c_int]
+            lib.oracle_attention_fwd_masked.restype = ctypes.c_int
             lib.oracle_attention_bwd.argtypes = [
                 dp, dp, dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_double, ctypes.c_int]
@@ -138,6 +147,53 @@ def attention(q, k, v, scale: float | None = None, causal: bool = False,
         rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), nr)
     if rc != 0:
         raise ValueError(f"oracle_attention_fwd failed ({rc})")
+    return o.reshape(lead + (nr, d)), lse.reshape(lead + (nr,))
+
+
+def attention_masked(q, k, v, scale: float | None = None, causal: bool = False,
+                     window=(-1, -1), alibi_slopes=None, rows=None):
+    """:func:`attention` with a local window and an ALiBi bias
+    (``oracle_attention_fwd_masked`` in ``fa_oracle.c``).
+
+    ``window = (left, right)``: key j is visible from query i iff
+    ``i - left <= j <= i + right`` (-1 = unbounded on that side), intersected
+    with the causal mask.  ``alibi_slopes``: one slope per head (``[H]``) or
+    None; the scaled score gets ``- slope[h] * |i - j|``.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have the same shape")
+    lead = q.shape[:-2]
+    N, d = q.shape[-2], q.shape[-1]
+    if q.ndim == 2:
+        B, H = 1, 1
+    elif q.ndim == 3:
+        B, H = q.shape[0], 1
+    elif q.ndim == 4:
+        B, H = q.shape[0], q.shape[1]
+    else:
+        raise ValueError("expected 2-D, 3-D or 4-D inputs")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    left, right = (int(window[0]), int(window[1]))
+    if left < -1 or right < -1:
+        raise ValueError("window sides must be >= -1")
+    slopes = None
+    if alibi_slopes is not None:
+        slopes = np.ascontiguousarray(np.asarray(alibi_slopes, dtype=np.float64).reshape(-1))
+        if slopes.size != H:
+            raise ValueError("alibi_slopes needs one slope per head")
+    rows_arr = np.arange(N, dtype=np.int32) if rows is None else np.ascontiguousarray(
+        np.asarray(rows, dtype=np.int32))
+    nr = int(rows_arr.size)
+    o = np.empty((B, H, nr, d), dtype=np.float64)
+    lse = np.empty((B, H, nr), dtype=np.float64)
+    rc = _load().oracle_attention_fwd_masked(
+        _dptr(q), _dptr(k), _dptr(v), _dptr(o), _dptr(lse), B, H, N, d, float(scale),
+        int(bool(causal)), left, right, None if slopes is None else _dptr(slopes),
+        rows_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), nr)
+    if rc != 0:
+        raise ValueError(f"oracle_attention_fwd_masked failed ({rc})")
     return o.reshape(lead + (nr, d)), lse.reshape(lead + (nr,))
 
 

@@ -30,3 +30,27 @@ def attention_fsum(q, k, v, scale=None, causal=False):
                   for c in range(d)])
         LSE.append(math.log(z))
     return O, LSE
+
+
+def attention_fsum_masked(q, k, v, scale=None, causal=False, window=(-1, -1), slope=0.0):
+    """:func:`attention_fsum` with a local window ``(left, right)`` (-1 =
+    unbounded) and an ALiBi bias ``-slope * |i - j|`` on the scaled scores,
+    one scalar at a time with ``math.fsum``.  Returns (O, LSE) lists."""
+    N = len(q)
+    d = len(q[0])
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    left, right = window
+    O, LSE = [], []
+    for i in range(N):
+        vis = [j for j in range(N)
+               if (left < 0 or j >= i - left) and (right < 0 or j <= i + right)
+               and (not causal or j <= i)]
+        s = [scale * math.fsum(float(q[i][c]) * float(k[j][c]) for c in range(d))
+             - slope * abs(i - j) for j in vis]
+        e = [math.exp(x) for x in s]
+        z = math.fsum(e)
+        O.append([math.fsum(e[n] * float(v[j][c]) for n, j in enumerate(vis)) / z
+                  for c in range(d)])
+        LSE.append(math.log(z))
+    return O, LSE

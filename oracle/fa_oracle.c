@@ -140,6 +140,84 @@ int oracle_attention_probs(const double *q, const double *k, int N, int d,
 }
 
 /*
+ * Forward with a local window and an ALiBi bias: the two masks the packed
+ * call of "Windows下RTX 3090编译Flash Attention 2.8.3全指南" (intelliparadigm.com)
+ * names as keyword arguments (window_size=(-1,-1), alibi_slopes, section
+ * 5.2 and 10.1) without defining them.  The reading taken:
+ *
+ *   key j visible from query i  iff  (left  < 0 || j >= i - left)
+ *                                 && (right < 0 || j <= i + right)
+ *                                 && (!causal  || j <= i)
+ *   s_ij = scale * q_i . k_j  -  slope[h] * |i - j|        (slopes may be NULL)
+ *
+ * then the same softmax, P V and logsumexp as oracle_attention_fwd.  The
+ * visible keys of a row form one range that always contains j = i.
+ * Layout and row subset as oracle_attention_fwd; slopes is [H] or NULL.
+ */
+int oracle_attention_fwd_masked(const double *q, const double *k, const double *v,
+                                double *o, double *lse, int B, int H, int N, int d,
+                                double scale, int causal, int left, int right,
+                                const double *slopes, const int *rows, int nrows)
+{
+    if (!q || !k || !v || !o || !rows) return -1;
+    if (B < 1 || H < 1 || N < 1 || d < 1 || nrows < 0) return -1;
+    for (int r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= N) return -1;
+    const long long total = (long long)B * H * nrows;
+    int failed = 0;
+
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!p) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (long long t = 0; t < total; ++t) {
+            if (!p) continue;
+            const long long bh = t / nrows;
+            const int h = (int)(bh % H);
+            const int r = (int)(t % nrows);
+            const int i = rows[r];
+            int lo = left < 0 ? 0 : i - left;
+            int hi = right < 0 ? N - 1 : i + right;
+            if (lo < 0) lo = 0;
+            if (hi > N - 1) hi = N - 1;
+            if (causal && hi > i) hi = i;
+            const double slope = slopes ? slopes[h] : 0.0;
+            const double *Q = q + (size_t)bh * N * d;
+            const double *K = k + (size_t)bh * N * d;
+            const double *V = v + (size_t)bh * N * d;
+            const double *qrow = Q + (size_t)i * d;
+            double *out = o + ((size_t)bh * nrows + r) * d;
+            double m = -INFINITY;
+            for (int j = lo; j <= hi; ++j) {
+                const double *krow = K + (size_t)j * d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += qrow[c] * krow[c];
+                p[j] = scale * dot - slope * fabs((double)(i - j));
+                if (p[j] > m) m = p[j];
+            }
+            double l = 0.0;
+            for (int j = lo; j <= hi; ++j) {
+                p[j] = exp(p[j] - m);
+                l += p[j];
+            }
+            for (int c = 0; c < d; ++c) out[c] = 0.0;
+            for (int j = lo; j <= hi; ++j) {
+                const double *vrow = V + (size_t)j * d;
+                for (int c = 0; c < d; ++c) out[c] += p[j] * vrow[c];
+            }
+            for (int c = 0; c < d; ++c) out[c] /= l;
+            if (lse) lse[(size_t)bh * nrows + r] = m + log(l);
+        }
+        free(p);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
  * Gradient of the forward above with respect to q, k and v, for an upstream
  * gradient dout of O (the logsumexp output is taken as not differentiated).
  * The pages name the backward pass only by its recomputation of the score
