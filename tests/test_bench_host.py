@@ -1,0 +1,57 @@
+"""Host-side logic of bench.py: FLOP and byte accounting, the traffic record's
+source-hash gate, the clock summary and its rejection rule.  No GPU."""
+import pytest
+
+import bench
+from exact_attention_154_b200 import synth
+
+
+def test_workload_flops_and_row_flops_agree():
+    w = synth.seqlen_sweep(1024, False)
+    assert w.flops == 4.0 * w.B * w.H * w.N ** 2 * w.d
+    assert bench.row_flops(w, range(w.N)) * w.B * w.H == pytest.approx(w.flops)
+    wc = synth.seqlen_sweep(1024, True)
+    # causal: row i sees i + 1 keys; the sum over rows is N (N + 1) / 2
+    full = bench.row_flops(wc, range(wc.N)) * wc.B * wc.H
+    assert full == pytest.approx(4.0 * wc.B * wc.H * wc.d * wc.N * (wc.N + 1) / 2)
+    assert bench.row_flops(wc, [0, 9]) == 4.0 * wc.d * (1 + 10)
+
+
+def test_algorithmic_bytes_of_the_bench_workload():
+    w = synth.seqlen_sweep(4096, False)
+    # q, k, v read and o written once in 16 bits, plus the fp32 LSE
+    assert bench.algorithmic_bytes(w) == 4 * 64 * 2 ** 20 + 4 * w.B * w.H * w.N
+
+
+def test_traffic_record_is_gated_by_the_source_hash(tmp_path, monkeypatch):
+    rec = tmp_path / "traffic.md"
+    rec.write_text(f"source_sha256: {bench.kernel_source_hash()}\n"
+                   "traffic_bytes_per_launch[sweep-n4096]: 123\n")
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(rec))
+    assert bench.profiled_traffic("sweep-n4096") == 123.0
+    assert bench.profiled_traffic("sweep-n8192") is None
+    rec.write_text("source_sha256: 0000000000000000\ntraffic_bytes_per_launch[sweep-n4096]: 123\n")
+    assert bench.profiled_traffic("sweep-n4096") is None
+    monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(tmp_path / "missing.md"))
+    assert bench.profiled_traffic("sweep-n4096") is None
+
+
+def test_clock_summary_and_rejection_rule():
+    s = bench.ClockSampler(0)
+    s.lines = [
+        "0, 1600, 1965, 990.1, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1650, 1965, 995.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1700, 1965, 980.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage",
+    ]
+    c = s.summary()
+    assert c == {"sm_mhz": 1650.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    assert bench.clocks_ok(c)  # the power cap is kept and noted
+    s.lines.append("0, 1200, 1965, 700.0, 0x8, Not Active, Active, Not Active, Not Active")
+    assert not bench.clocks_ok(s.summary())  # a thermal slowdown rejects the run
+
+
+def test_peaks_fall_back_when_the_measured_file_is_missing(monkeypatch, tmp_path):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.load_peaks()
+    assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
