@@ -340,12 +340,8 @@ def bench_gpu(args, w, key, world, rank, local):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": synth.DTYPE_NAME[w.dtype], "data": "synthetic (seeded randn, see DESIGN.md)",
-        "config": dict(w.describe(), workload_key=key,
-                       parallelism=f"replicas{world}" if world > 1 else "single-gpu",
-                       global_batch=w.B * world, seq_len=w.N,
-                       l2="inputs larger than L2 (q,k,v,o = %d MiB per step)" %
-                          ((4 if w.layout != "packed" else 0) * w.B * w.H * w.N * w.d * 2 >> 20)),
+        "dtype": synth.DTYPE_NAME[w.dtype], "data": DATA,
+        "config": run_config(w, key, world),
         "pct_of_peak": {
             "measured_burst": round(100 * achieved / peaks["bf16_tflops"], 2),
             "measured_sustained": round(100 * achieved / peaks["bf16_tflops_sustained"], 2),
@@ -438,7 +434,7 @@ def bench_gpu_bwd(args, w, key, world, rank, local):
         "metric": METRIC_BWD, "value": round(world * achieved, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": synth.DTYPE_NAME[w.dtype], "data": "synthetic (seeded randn, see DESIGN.md)",
+        "dtype": synth.DTYPE_NAME[w.dtype], "data": DATA,
         "config": dict(w.describe(), workload_key=key, direction="bwd",
                        parallelism=f"replicas{world}" if world > 1 else "single-gpu",
                        global_batch=w.B * world, seq_len=w.N,
@@ -486,6 +482,26 @@ def cpu_oracle_bwd_sample(w, host, target_s=12.0):
                       f"fp64 gradient oracle, one head per host thread"}
 
 
+L2_BYTES = 126 * 10 ** 6
+DATA = "synthetic: seeded CPU torch randn (fp32) x sigma, rounded once to the compute dtype"
+
+
+def run_config(w, key, world):
+    """The ``config`` object of a forward line; both arms print the same one."""
+    return dict(w.describe(), workload_key=key,
+                parallelism=f"replicas{world}" if world > 1 else "single-gpu",
+                global_batch=w.B * world, seq_len=w.N,
+                l2=l2_note(4 * w.B * w.H * w.N * w.d * 2))
+
+
+def l2_note(step_bytes):
+    """How the timed steps relate to the 126 MB L2 (no flush is done)."""
+    if step_bytes > L2_BYTES:
+        return "inputs larger than L2 (q,k,v,o = %d MiB per step)" % (step_bytes >> 20)
+    return "inputs fit in L2 (q,k,v,o = %d KiB per step; no flush between steps)" % (
+        step_bytes >> 10)
+
+
 def algorithmic_bytes(w):
     e = 2
     return 4 * w.B * w.H * w.N * w.d * e + 4 * w.B * w.H * w.N
@@ -522,8 +538,8 @@ def main():
         line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic (seeded randn)",
-                "config": dict(w.describe(), workload_key=args.workload),
+                "dtype": "f64", "data": DATA,
+                "config": run_config(w, args.workload, args.gpus),
                 "cpu_baseline": dict(info, value=round(value, 6)),
                 "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0},

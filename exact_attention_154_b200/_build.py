@@ -10,7 +10,11 @@ CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libfa_sm100.so")
 SOURCES = ["fa_api.cu"]
-HEADERS = ["fa_fwd_sm100.cuh", "sm100_ptx.cuh"]
+
+
+def headers():
+    """Every header under csrc/: a change to any of them rebuilds the library."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith((".cuh", ".h")))
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
@@ -27,7 +31,7 @@ def nvcc_path() -> str:
 
 
 def _inputs():
-    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    files = [os.path.join(CSRC, f) for f in SOURCES + headers()]
     files.append(os.path.join(ROOT, "include", "fa.h"))
     return files
 

@@ -85,6 +85,26 @@ def _stream_ptr(t: torch.Tensor):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
 
 
+def same_device(named) -> torch.device:
+    """The one device every ``(name, tensor)`` pair lives on; raises if they differ.
+
+    The library resolves its per-device state (SM count, kernel attributes, the
+    backward's scratch array) from the *current* device, so every call runs
+    with the tensors' device made current (see :func:`_on`)."""
+    dev = None
+    for name, t in named:
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev}")
+    return dev
+
+
+def _on(dev: torch.device):
+    """Context that makes ``dev`` the current CUDA device for one library call."""
+    return torch.cuda.device(dev)
+
+
 def _check_tensor(t: torch.Tensor, name: str):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
@@ -128,9 +148,12 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None =
         lse_ptr = lse.data_ptr()
     else:
         lse = None
-    rc = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
-                       B, H, N, d, 0.0 if scale is None else float(scale), int(bool(causal)),
-                       _DT[q.dtype], _stream_ptr(q))
+    dev = same_device([("q", q), ("k", k), ("v", v), ("out", out)] +
+                      ([("lse", lse)] if lse is not None else []))
+    with _on(dev):
+        rc = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
+                           B, H, N, d, 0.0 if scale is None else float(scale),
+                           int(bool(causal)), _DT[q.dtype], _stream_ptr(q))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd")
     return out, lse
@@ -148,11 +171,15 @@ def fwd_qkvpacked(qkv: torch.Tensor, dropout_p: float = 0.0, softmax_scale: floa
         out = torch.empty((B, N, H, d), device=qkv.device, dtype=qkv.dtype)
     else:
         _check_tensor(out, "out")
+    if out.shape != (B, N, H, d) or out.dtype != qkv.dtype:
+        raise ValueError("out must be [B, N, H, d] in qkv's dtype")
     lse = torch.empty((B, H, N), device=qkv.device, dtype=torch.float32) if return_lse else None
-    rc = load().fa_fwd_qkvpacked(
-        qkv.data_ptr(), out.data_ptr(), None if lse is None else lse.data_ptr(), B, N, H, d,
-        0.0 if softmax_scale is None else float(softmax_scale), int(bool(causal)),
-        float(dropout_p), _DT[qkv.dtype], _stream_ptr(qkv))
+    dev = same_device([("qkv", qkv), ("out", out)])
+    with _on(dev):
+        rc = load().fa_fwd_qkvpacked(
+            qkv.data_ptr(), out.data_ptr(), None if lse is None else lse.data_ptr(), B, N, H, d,
+            0.0 if softmax_scale is None else float(softmax_scale), int(bool(causal)),
+            float(dropout_p), _DT[qkv.dtype], _stream_ptr(qkv))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_qkvpacked")
     return out, lse
@@ -176,11 +203,13 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous [B, H, N] float32 tensor")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dev = same_device([("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("dout", dout)])
     work = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
-    rc = load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                       dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), work.data_ptr(),
-                       B, H, N, d, 0.0 if scale is None else float(scale), int(bool(causal)),
-                       _DT[q.dtype], _stream_ptr(q))
+    with _on(dev):
+        rc = load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                           work.data_ptr(), B, H, N, d, 0.0 if scale is None else float(scale),
+                           int(bool(causal)), _DT[q.dtype], _stream_ptr(q))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv
@@ -201,10 +230,13 @@ def bwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tens
     if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous [B, H, N] float32 tensor")
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    rc = load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                               lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                               dv.data_ptr(), B, H, N, d, 0.0 if scale is None else float(scale),
-                               int(bool(causal)), _DT[q.dtype], _stream_ptr(q))
+    dev = same_device([("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("dout", dout)])
+    with _on(dev):
+        rc = load().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                   dv.data_ptr(), B, H, N, d,
+                                   0.0 if scale is None else float(scale), int(bool(causal)),
+                                   _DT[q.dtype], _stream_ptr(q))
     if rc != FA_OK:
         raise FaError(rc, "fa_bwd_noalloc")
     return dq, dk, dv

@@ -91,7 +91,6 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
 int fa_fwd_qkvpacked(const void *qkv, void *o, float *lse, int B, int N, int H, int d, float scale,
                      int causal, float dropout_p, int dtype, struct CUstream_st *stream);
 
-/* Static text for a status code. */
 /*
  * Gradient of fa_fwd: dQ, dK, dV for an upstream gradient dO of O.  The score
  * tile is recomputed from q, k and the forward's logsumexp, the
@@ -134,6 +133,7 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, c
                    const void *dout, void *dq, void *dk, void *dv, int B, int H, int N, int d,
                    float scale, int causal, int dtype, struct CUstream_st *stream);
 
+/* Static text for a status code. */
 const char *fa_strerror(int status);
 
 /*
