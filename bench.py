@@ -54,6 +54,9 @@ def workloads_by_key():
         "packed-b2-n256-h12": synth.packed_qkv_b2_n256_h12(),
         "causal-h128-n2048": synth.many_heads_causal_n2048(),
         "hd256-causal-n8192": synth.headdim256_causal(),
+        "window256-causal-n4096": synth.window_causal_n4096(),
+        "alibi-causal-n4096": synth.alibi_causal_n4096(),
+        "varlen-mix-causal": synth.varlen_mix_causal(),
     }
     for n in synth.SWEEP_N:
         table[f"sweep-n{n}"] = synth.seqlen_sweep(n, False)
@@ -182,8 +185,40 @@ def device_inputs(w):
     return tuple(t.cuda() for t in synth.make_inputs(w))
 
 
+def tokens(w):
+    return int(sum(w.lengths)) if w.layout == "varlen" else w.B * w.N
+
+
 def launcher(w, dev_inputs):
     """Returns a zero-argument callable issuing one forward on the current stream."""
+    lib = fa.load()
+    slopes = synth.alibi_slopes(w.H).cuda() if w.alibi else None
+    sp = None if slopes is None else slopes.data_ptr()
+    if w.layout == "varlen":
+        q, k, v, cu = dev_inputs
+        out = torch.empty_like(q)
+        lse = torch.empty((w.H, q.shape[0]), device="cuda", dtype=torch.float32)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                cu.data_ptr(), w.B, w.N, q.shape[0], w.H, w.d, 0.0, int(w.causal), w.window[0],
+                w.window[1], sp, w.dtype)
+
+        def go():
+            rc = lib.fa_fwd_varlen(*args, torch.cuda.current_stream().cuda_stream)
+            if rc:
+                raise fa.FaError(rc, "fa_fwd_varlen")
+        return go, (out, lse, slopes)
+    if w.masked and w.layout == "bhnd":
+        q, k, v = dev_inputs
+        out = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), device="cuda", dtype=torch.float32)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B,
+                w.H, w.N, w.d, 0.0, int(w.causal), w.window[0], w.window[1], sp, w.dtype)
+
+        def go():
+            rc = lib.fa_fwd_ext(*args, torch.cuda.current_stream().cuda_stream)
+            if rc:
+                raise fa.FaError(rc, "fa_fwd_ext")
+        return go, (out, lse, slopes)
     if w.layout == "packed":
         (qkv,) = dev_inputs
         out = torch.empty((w.B, w.N, w.H, w.d), device="cuda", dtype=qkv.dtype)
@@ -239,14 +274,21 @@ def time_e2e(w, steps, warmup, world):
         o_host = torch.empty_like(host[0]).pin_memory()
     lse_host = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
     stream = torch.cuda.current_stream()
+    slopes = synth.alibi_slopes(w.H).cuda() if w.alibi else None
+    if w.layout == "varlen":
+        lse_host = torch.empty((w.H, host[0].shape[0]), dtype=torch.float32).pin_memory()
 
     def step():
         for h, d in zip(host, dev):
             d.copy_(h, non_blocking=True)
         if w.layout == "packed":
             o, lse = fa.fwd_qkvpacked(dev[0], causal=w.causal)
+        elif w.layout == "varlen":
+            o, lse = fa.fwd_varlen(dev[0], dev[1], dev[2], dev[3], w.N, causal=w.causal,
+                                   window_size=w.window, alibi_slopes=slopes)
         else:
-            o, lse = fa.fwd(dev[0], dev[1], dev[2], causal=w.causal)
+            o, lse = fa.fwd(dev[0], dev[1], dev[2], causal=w.causal, window_size=w.window,
+                            alibi_slopes=slopes)
         o_host.copy_(o, non_blocking=True)
         lse_host.copy_(lse, non_blocking=True)
 
@@ -269,6 +311,13 @@ def time_e2e(w, steps, warmup, world):
 
 def row_flops(w, rows):
     """Algorithmic FLOPs of the given query rows (4*d per visible key)."""
+    if w.window != (-1, -1):
+        left, right = w.window
+        right = 0 if w.causal else right
+        r = np.asarray(rows, dtype=np.int64)
+        lo = np.zeros_like(r) if left < 0 else np.maximum(r - left, 0)
+        hi = np.full_like(r, w.N - 1) if right < 0 else np.minimum(r + right, w.N - 1)
+        return float(4.0 * w.d * (hi - lo + 1).sum())
     if w.causal:
         return float(sum(4.0 * w.d * (int(r) + 1) for r in rows))
     return 4.0 * w.d * w.N * len(rows)
@@ -285,29 +334,58 @@ class OracleSampler:
         self.oracle, self.w = oracle, w
         if w.layout == "packed":
             q, k, v = synth.unpack_qkv(synth.make_inputs(w)[0])
+        elif w.layout == "varlen":
+            q, k, v, cu = synth.make_inputs(w)
+            self.cu = cu.numpy()
         else:
             q, k, v = synth.make_inputs(w)
         self.qkv = tuple(t.double().numpy() for t in (q, k, v))
         self.rng = np.random.default_rng(w.seed + 2000)
         self.scale = fa.default_scale(w.d)
+        self.slopes = synth.alibi_slopes(w.H).double().numpy() if w.alibi else None
+        if w.layout == "varlen":
+            # whole sequences, shortest first, until about target_s of work
+            dt, fl, _ = self.run(1)
+            self.nseq = max(1, min(w.B, int(max(target_s, 1e-3) / max(dt, 1e-4))))
+            return
         n0 = min(w.N, 2)
         dt, _, _ = self.run(n0)
         self.nrows = max(1, min(w.N, int(n0 * max(target_s, 1e-3) / max(dt, 1e-4))))
 
-    def run(self, nrows):
+    def run(self, n):
         w = self.w
-        rows = np.sort(self.rng.choice(w.N, size=nrows, replace=False)).astype(np.int32)
+        if w.layout == "varlen":
+            order = np.argsort(np.diff(self.cu), kind="stable")[:n]
+            t0 = time.perf_counter()
+            fl = 0.0
+            for b in order:
+                s0, s1 = int(self.cu[b]), int(self.cu[b + 1])
+                self.oracle.attention_varlen(*(t[s0:s1] for t in self.qkv), [0, s1 - s0],
+                                             scale=self.scale, causal=w.causal, window=w.window,
+                                             alibi_slopes=self.slopes)
+                fl += 4.0 * w.d * w.H * synth.visible_pairs(s1 - s0, w.causal, w.window)
+            return time.perf_counter() - t0, fl, n
+        rows = np.sort(self.rng.choice(w.N, size=n, replace=False)).astype(np.int32)
         t0 = time.perf_counter()
-        self.oracle.attention(*self.qkv, scale=self.scale, causal=w.causal, rows=rows)
-        return time.perf_counter() - t0, row_flops(w, rows) * w.B * w.H, nrows
+        if w.masked:
+            self.oracle.attention_masked(*self.qkv, scale=self.scale, causal=w.causal, rows=rows,
+                                         window=w.window, alibi_slopes=self.slopes)
+        else:
+            self.oracle.attention(*self.qkv, scale=self.scale, causal=w.causal, rows=rows)
+        return time.perf_counter() - t0, row_flops(w, rows) * w.B * w.H, n
 
     def step(self):
-        dt, fl, nrows = self.run(self.nrows)
         w = self.w
+        if w.layout == "varlen":
+            dt, fl, n = self.run(self.nseq)
+            sample = (f"the {n} shortest of the {w.B} sequences of the workload, whole, "
+                      f"fp64 oracle, all host threads")
+        else:
+            dt, fl, n = self.run(self.nrows)
+            sample = (f"{n} seeded query rows in each of the {w.B * w.H} (b, h) heads of "
+                      f"the workload (of N={w.N}), fp64 oracle, all host threads")
         return {"value": fl / dt / 1e12, "unit": UNIT, "cores": self.oracle.num_threads(),
-                "kind": "oracle", "seconds": round(dt, 4),
-                "sample": f"{nrows} seeded query rows in each of the {w.B * w.H} (b, h) heads of "
-                          f"the workload (of N={w.N}), fp64 oracle, all host threads"}
+                "kind": "oracle", "seconds": round(dt, 4), "sample": sample}
 
 
 def cpu_oracle_sample(w, target_s=12.0):
@@ -491,7 +569,7 @@ def run_config(w, key, world):
     return dict(w.describe(), workload_key=key,
                 parallelism=f"replicas{world}" if world > 1 else "single-gpu",
                 global_batch=w.B * world, seq_len=w.N,
-                l2=l2_note(4 * w.B * w.H * w.N * w.d * 2))
+                l2=l2_note(4 * tokens(w) * w.H * w.d * 2))
 
 
 def l2_note(step_bytes):
@@ -504,7 +582,7 @@ def l2_note(step_bytes):
 
 def algorithmic_bytes(w):
     e = 2
-    return 4 * w.B * w.H * w.N * w.d * e + 4 * w.B * w.H * w.N
+    return 4 * tokens(w) * w.H * w.d * e + 4 * tokens(w) * w.H
 
 
 def main():

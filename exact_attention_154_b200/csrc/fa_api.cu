@@ -16,7 +16,7 @@ namespace {
 
 using namespace fa_sm100;
 
-constexpr int kVersion = 1 * 10000 + 1 * 100 + 0;  // 1.1.0: the backward entry points
+constexpr int kVersion = 1 * 10000 + 2 * 100 + 0;  // 1.2.0: local window, ALiBi, varlen
 // Limit of every mbarrier wait of the kernel (2 s unless the build sets it).
 #ifndef FA_WAIT_LIMIT_NS
 #define FA_WAIT_LIMIT_NS 2000000000ull
@@ -41,7 +41,7 @@ struct DeviceState {
   bool ready = false;
   bool is_sm100 = false;
   int sm_count = 0;
-  bool attr_set[6] = {false, false, false, false, false, false};
+  bool attr_set[12] = {};
   bool bwd_attr_set[8] = {false, false, false, false, false, false, false, false};
   float* bwd_scratch = nullptr;  // this device's g_bwd_scratch
 };
@@ -110,12 +110,12 @@ template <> struct Pick<256> { static constexpr int QS = 1, KVS = 2; };
 
 int q_tiles_for(int d) { return d == 256 ? 1 : 2; }
 
-template <int HD, bool BF16>
+template <int HD, bool BF16, bool ALIBI>
 int launch(FwdParams& p, DeviceState& st, cudaStream_t stream) {
   constexpr int QS = Pick<HD>::QS, KVS = Pick<HD>::KVS;
   using C = FwdCfg<HD, QS, KVS, BF16>;
-  auto kernel = fa_fwd_kernel<HD, QS, KVS, BF16>;
-  const int slot = (HD == 64 ? 0 : HD == 128 ? 2 : 4) + (BF16 ? 1 : 0);
+  auto kernel = fa_fwd_kernel<HD, QS, KVS, BF16, ALIBI>;
+  const int slot = (HD == 64 ? 0 : HD == 128 ? 2 : 4) + (BF16 ? 1 : 0) + (ALIBI ? 6 : 0);
   if (!st.attr_set[slot]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess) {
@@ -132,6 +132,16 @@ int launch(FwdParams& p, DeviceState& st, cudaStream_t stream) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Local window sides: -1 (unbounded) or >= 0; a side that reaches past the
+// longest sequence is unbounded; with the causal mask the right side is 0.
+int normalize_window(int N, int causal, int* left, int* right) {
+  if (*left < -1 || *right < -1) return FA_ERR_ARG;
+  if (*left >= N) *left = -1;
+  if (*right >= N) *right = -1;
+  if (causal) *right = 0;
+  return FA_OK;
+}
+
 int check_common(int B, int H, int N, int d, float* scale, int causal, int dtype) {
   if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
@@ -147,9 +157,30 @@ int check_common(int B, int H, int N, int d, float* scale, int causal, int dtype
   return FA_OK;
 }
 
-int run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-        int d, float scale, int causal, int dtype, long long sn, long long sh, long long sb,
-        long long osn, long long osh, long long osb, cudaStream_t stream) {
+// One forward problem as the kernel sees it: operand views, output layout,
+// masks.  Strides are in elements.
+struct Problem {
+  const void *q, *k, *v;
+  void* o;
+  float* lse;
+  int B, H, N, d;  // N: sequence length (the longest one when cu_seqlens is set)
+  float scale;
+  int causal, dtype;
+  long long sn, sh, sb;     // q / k / v: row, head, batch
+  long long osn, osh, osb;  // o
+  long long lsb, lsh;       // lse: batch, head (rows are contiguous)
+  int map_rows, map_batches;
+  int window_left, window_right;
+  const float* alibi;
+  const int* cu_seqlens;
+};
+
+template <int HD, bool BF16>
+int launch_masks(FwdParams& p, bool alibi, DeviceState& st, cudaStream_t stream) {
+  return alibi ? launch<HD, BF16, true>(p, st, stream) : launch<HD, BF16, false>(p, st, stream);
+}
+
+int run(const Problem& pr, cudaStream_t stream) {
   std::lock_guard<std::mutex> lock(g_mutex);
   int rc = get_encode_fn();
   if (rc != FA_OK) return rc;
@@ -159,31 +190,87 @@ int run(const void* q, const void* k, const void* v, void* o, float* lse, int B,
 
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
-  if ((rc = encode_operand(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
-  p.o = o;
-  p.lse = lse;
-  p.o_stride_n = osn;
-  p.o_stride_h = osh;
-  p.o_stride_b = osb;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.causal = causal;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  const int rows_per_tile = 128 * q_tiles_for(d);
-  p.num_qblocks = (N + rows_per_tile - 1) / rows_per_tile;
-  p.num_tiles = B * H * p.num_qblocks;
+  const int R = pr.map_rows, NB = pr.map_batches;
+  if ((rc = encode_operand(&p.tmap_q, pr.q, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
+                           128)) != FA_OK)
+    return rc;
+  if ((rc = encode_operand(&p.tmap_k, pr.k, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
+                           128)) != FA_OK)
+    return rc;
+  if ((rc = encode_operand(&p.tmap_v, pr.v, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
+                           128)) != FA_OK)
+    return rc;
+  p.o = pr.o;
+  p.lse = pr.lse;
+  p.o_stride_n = pr.osn;
+  p.o_stride_h = pr.osh;
+  p.o_stride_b = pr.osb;
+  p.lse_stride_b = pr.lsb;
+  p.lse_stride_h = pr.lsh;
+  p.B = pr.B;
+  p.H = pr.H;
+  p.N = pr.N;
+  p.rows_total = R;
+  p.cu_seqlens = pr.cu_seqlens;
+  p.causal = pr.causal;
+  p.window_left = pr.window_left;
+  p.window_right = pr.window_right;
+  p.alibi_slopes = pr.alibi;
+  p.scale_log2 = pr.scale * 1.4426950408889634f;
+  const int rows_per_tile = 128 * q_tiles_for(pr.d);
+  p.num_qblocks = (pr.N + rows_per_tile - 1) / rows_per_tile;
+  p.num_tiles = pr.B * pr.H * p.num_qblocks;
   p.wait_limit_ns = kWaitLimitNs;
 
-  const bool bf16 = dtype == FA_BF16;
-  switch (d) {
-    case 64: return bf16 ? launch<64, true>(p, *st, stream) : launch<64, false>(p, *st, stream);
-    case 128: return bf16 ? launch<128, true>(p, *st, stream) : launch<128, false>(p, *st, stream);
-    default: return bf16 ? launch<256, true>(p, *st, stream) : launch<256, false>(p, *st, stream);
+  const bool bf16 = pr.dtype == FA_BF16, alibi = pr.alibi != nullptr;
+  switch (pr.d) {
+    case 64:
+      return bf16 ? launch_masks<64, true>(p, alibi, *st, stream)
+                  : launch_masks<64, false>(p, alibi, *st, stream);
+    case 128:
+      return bf16 ? launch_masks<128, true>(p, alibi, *st, stream)
+                  : launch_masks<128, false>(p, alibi, *st, stream);
+    default:
+      return bf16 ? launch_masks<256, true>(p, alibi, *st, stream)
+                  : launch_masks<256, false>(p, alibi, *st, stream);
   }
 }
+
+// [B, H, N, d] operands and output, [B, H, N] logsumexp.
+Problem bhnd_problem(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int N, int d, float scale, int causal, int dtype) {
+  Problem pr;
+  std::memset(&pr, 0, sizeof(pr));
+  pr.q = q; pr.k = k; pr.v = v; pr.o = o; pr.lse = lse;
+  pr.B = B; pr.H = H; pr.N = N; pr.d = d; pr.scale = scale; pr.causal = causal; pr.dtype = dtype;
+  pr.sn = pr.osn = d;
+  pr.sh = pr.osh = (long long)N * d;
+  pr.sb = pr.osb = (long long)H * N * d;
+  pr.lsb = (long long)H * N;
+  pr.lsh = N;
+  pr.map_rows = N;
+  pr.map_batches = B;
+  pr.window_left = pr.window_right = -1;
+  return pr;
+}
+
+// qkv [B, N, 3, H, d] (q / k / v differ by H * d elements), o [B, N, H, d].
+Problem packed_problem(const void* qkv, void* o, float* lse, int B, int N, int H, int d,
+                       float scale, int causal, int dtype) {
+  const char* base = static_cast<const char*>(qkv);
+  const long long hd = (long long)H * d;
+  Problem pr = bhnd_problem(base, base + 2 * hd, base + 4 * hd, o, lse, B, H, N, d, scale, causal,
+                            dtype);
+  pr.sn = 3 * hd;
+  pr.sh = d;
+  pr.sb = (long long)N * 3 * hd;
+  pr.osn = hd;
+  pr.osh = d;
+  pr.osb = (long long)N * hd;
+  return pr;
+}
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 template <int HD, bool BF16, bool KV>
 int launch_bwd_kernel(const BwdParams& p, DeviceState& st, cudaStream_t stream) {
@@ -216,33 +303,78 @@ int launch_bwd(const BwdParams& p, DeviceState& st, cudaStream_t stream) {
 
 extern "C" {
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
-           int d, float scale, int causal, int dtype, struct CUstream_st* stream) {
+int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int N, int d, float scale, int causal, int window_left, int window_right,
+               const float* alibi_slopes, int dtype, struct CUstream_st* stream) {
   if (!q || !k || !v || !o) return FA_ERR_ARG;
   int rc = check_common(B, H, N, d, &scale, causal, dtype);
   if (rc != FA_OK) return rc;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+  if ((rc = normalize_window(N, causal, &window_left, &window_right)) != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !aligned4(alibi_slopes))
     return FA_ERR_ALIGN;
-  const long long sn = d, sh = (long long)N * d, sb = (long long)H * N * d;
-  return run(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, sn, sh, sb, sn, sh, sb,
-             reinterpret_cast<cudaStream_t>(stream));
+  Problem pr = bhnd_problem(q, k, v, o, lse, B, H, N, d, scale, causal, dtype);
+  pr.window_left = window_left;
+  pr.window_right = window_right;
+  pr.alibi = alibi_slopes;
+  return run(pr, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int N, int H, int d, float scale,
-                     int causal, float dropout_p, int dtype, struct CUstream_st* stream) {
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N,
+           int d, float scale, int causal, int dtype, struct CUstream_st* stream) {
+  return fa_fwd_ext(q, k, v, o, lse, B, H, N, d, scale, causal, -1, -1, nullptr, dtype, stream);
+}
+
+int fa_fwd_qkvpacked_ext(const void* qkv, void* o, float* lse, int B, int N, int H, int d,
+                         float scale, int causal, float dropout_p, int window_left,
+                         int window_right, const float* alibi_slopes, int dtype,
+                         struct CUstream_st* stream) {
   if (!qkv || !o) return FA_ERR_ARG;
   if (!(dropout_p == 0.0f)) return std::isnan(dropout_p) ? FA_ERR_ARG : FA_ERR_UNSUPPORTED;
   int rc = check_common(B, H, N, d, &scale, causal, dtype);
   if (rc != FA_OK) return rc;
-  if (!aligned16(qkv) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+  if ((rc = normalize_window(N, causal, &window_left, &window_right)) != FA_OK) return rc;
+  if (!aligned16(qkv) || !aligned16(o) || !aligned4(lse) || !aligned4(alibi_slopes))
     return FA_ERR_ALIGN;
-  // qkv [B, N, 3, H, d]: q/k/v differ by H*d elements; o is [B, N, H, d].
-  const char* base = static_cast<const char*>(qkv);
-  const long long hd = (long long)H * d;
-  const long long sn = 3 * hd, sh = d, sb = (long long)N * 3 * hd;
-  return run(base, base + 2 * hd, base + 4 * hd, o, lse, B, H, N, d, scale, causal, dtype, sn, sh,
-             sb, hd, d, (long long)N * hd, reinterpret_cast<cudaStream_t>(stream));
+  Problem pr = packed_problem(qkv, o, lse, B, N, H, d, scale, causal, dtype);
+  pr.window_left = window_left;
+  pr.window_right = window_right;
+  pr.alibi = alibi_slopes;
+  return run(pr, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int N, int H, int d, float scale,
+                     int causal, float dropout_p, int dtype, struct CUstream_st* stream) {
+  return fa_fwd_qkvpacked_ext(qkv, o, lse, B, N, H, d, scale, causal, dropout_p, -1, -1, nullptr,
+                              dtype, stream);
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens, int batch, int max_seqlen, int total, int H, int d,
+                  float scale, int causal, int window_left, int window_right,
+                  const float* alibi_slopes, int dtype, struct CUstream_st* stream) {
+  if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_ARG;
+  int rc = check_common(batch, H, max_seqlen, d, &scale, causal, dtype);
+  if (rc != FA_OK) return rc;
+  if (total < 1 || (long long)total * H * d > (1ll << 46)) return FA_ERR_ARG;
+  if ((rc = normalize_window(max_seqlen, causal, &window_left, &window_right)) != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse) ||
+      !aligned4(alibi_slopes) || !aligned4(cu_seqlens))
+    return FA_ERR_ALIGN;
+  // q, k, v, o [total, H, d]; lse [H, total]; one tensor-map batch
+  Problem pr = bhnd_problem(q, k, v, o, lse, batch, H, max_seqlen, d, scale, causal, dtype);
+  pr.sn = pr.osn = (long long)H * d;
+  pr.sh = pr.osh = d;
+  pr.sb = pr.osb = (long long)total * H * d;
+  pr.lsb = 0;
+  pr.lsh = total;
+  pr.map_rows = total;
+  pr.map_batches = 1;
+  pr.window_left = window_left;
+  pr.window_right = window_right;
+  pr.alibi = alibi_slopes;
+  pr.cu_seqlens = cu_seqlens;
+  return run(pr, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -350,6 +482,7 @@ const char* fa_strerror(int status) {
     case FA_ERR_UNSUPPORTED: return "unsupported option (dropout_p must be 0)";
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "kernel gave up on a bounded wait";
+    case FA_ERR_SEQLENS: return "cu_seqlens out of range (seen by the kernel)";
     case FA_ERR_DEVICE: return "current device is not sm_100";
     default: return "unknown status";
   }
@@ -373,7 +506,8 @@ int fa_device_status(int clear, unsigned int* detail) {
     }
   }
   if (detail) *detail = word;
-  return word ? FA_ERR_TIMEOUT : FA_OK;
+  if (word == 0) return FA_OK;
+  return (word >> 8) == kRoleArgs ? FA_ERR_SEQLENS : FA_ERR_TIMEOUT;
 }
 
 int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st* stream) {

@@ -76,21 +76,36 @@ __device__ unsigned int g_fa_watchdog = 0u;
 enum WaitSite : unsigned {
   kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteQFull = 3, kSiteKvFull = 4, kSitePFull = 5,
   kSiteSFull = 6, kSiteODone = 7, kSiteSelfTest = 8, kSiteDrain = 9, kSiteSFree = 10,
-  kSitePFree = 11, kSiteAlign = 12, kSiteXch = 13
+  kSitePFree = 11, kSiteAlign = 12, kSiteXch = 13, kSiteSeqlens = 14
 };
-enum Role : unsigned { kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4 };
+// kRoleArgs: not a wait but a device-side argument check (cu_seqlens out of
+// range); the offending work tile is skipped.
+enum Role : unsigned {
+  kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4, kRoleArgs = 5
+};
 
 struct FwdParams {
-  CUtensorMap tmap_q;  // 4-D (d, N, H, B) views of q, k, v; box 64 elements x 128 rows
+  // 4-D (d, rows, H, batches) views of q, k, v; box 64 elements x 128 rows.
+  // Fixed-length problems: rows = N, batches = B.  Variable-length problems
+  // (cu_seqlens != nullptr): rows = the packed token count, one batch.
+  CUtensorMap tmap_q;
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   void* o;
-  float* lse;  // [B, H, N] or nullptr
+  float* lse;  // nullptr, or indexed [bc * lse_stride_b + h * lse_stride_h + token row]
   long long o_stride_b, o_stride_h, o_stride_n;  // in elements
-  int B, H, N;
+  long long lse_stride_b, lse_stride_h;
+  int B, H, N;       // N: the sequence length, or the longest one when variable
+  int rows_total;    // rows of the tensor maps (N, or the packed token count)
+  const int* cu_seqlens;  // [B + 1] token offsets of the sequences, or nullptr
   int causal;
+  // Key j is visible from query i iff i - window_left <= j <= i + window_right
+  // (and j < the sequence length); -1 leaves that side unbounded.  The causal
+  // mask arrives here as window_right = 0.
+  int window_left, window_right;
+  const float* alibi_slopes;  // [H]: the scaled score gets -slope[h] * |i - j|; or nullptr
   float scale_log2;  // scale * log2(e)
-  int num_qblocks;   // query blocks per (b, h)
+  int num_qblocks;   // query blocks per (b, h) (of the longest sequence)
   int num_tiles;     // B * H * num_qblocks
   unsigned long long wait_limit_ns;
 };
@@ -169,16 +184,36 @@ struct FwdCfg {
   static_assert(128 * QS <= 256 && 256 + QS * HD <= 512, "TMEM budget");
 };
 
+// One work tile: up to two 128-row Q tiles of one (sequence, head).  Q tile s
+// needs the key blocks [lo[s], hi[s]) (empty: lo == hi == 0); the work tile
+// streams their union [lo_u, lo_u + n_u), which is contiguous because the Q
+// tiles are adjacent and every row sees its own key.
 struct TileInfo {
-  int b, h, q0, n[2], n_max;
+  int b, h, q0;  // q0: first query row, relative to the sequence
+  int len;       // the sequence's length (queries = keys)
+  int row0;      // tensor-map row of the sequence's first token
+  int bc;        // tensor-map batch coordinate
+  int lo[2], hi[2];
+  int lo_u, n_u;
 };
 
-// Key blocks a 128-row Q tile starting at row r0 needs: all of them, or with
-// the causal mask those up to and including its diagonal.
-__device__ __forceinline__ int key_blocks(const FwdParams& p, int r0) {
-  const int nkv = (p.N + BN - 1) / BN;
-  if (r0 >= p.N) return 0;
-  return p.causal ? min(nkv, r0 / BN + 1) : nkv;
+__device__ __forceinline__ bool in_range(const TileInfo& ti, int s, int j) {
+  return j >= ti.lo[s] && j < ti.hi[s];
+}
+
+// Key blocks [lo, hi) a 128-row Q tile starting at row r0 of a sequence of
+// `len` tokens needs: those holding a key visible from one of its rows (up to
+// and including the diagonal block with the causal mask, the blocks the window
+// reaches with a local window).
+__device__ __forceinline__ void key_range(const FwdParams& p, int len, int r0, int& lo, int& hi) {
+  if (r0 >= len) {
+    lo = hi = 0;
+    return;
+  }
+  const int nkv = (len + BN - 1) / BN;
+  const int last_row = min(r0 + BM - 1, len - 1);
+  lo = p.window_left < 0 ? 0 : max(0, r0 - p.window_left) / BN;
+  hi = p.window_right < 0 ? nkv : min(len - 1, last_row + p.window_right) / BN + 1;
 }
 
 template <int QS>
@@ -201,9 +236,28 @@ __device__ __forceinline__ TileInfo decode_tile(const FwdParams& p, int t) {
   ti.b = bh / p.H;
   ti.h = bh - ti.b * p.H;
   ti.q0 = qblock * BM * QS;
-  ti.n[0] = key_blocks(p, ti.q0);
-  ti.n[1] = QS == 2 ? key_blocks(p, ti.q0 + BM) : 0;
-  ti.n_max = max(ti.n[0], ti.n[1]);
+  if (p.cu_seqlens != nullptr) {
+    const int s0 = __ldg(p.cu_seqlens + ti.b), s1 = __ldg(p.cu_seqlens + ti.b + 1);
+    ti.row0 = s0;
+    ti.len = s1 - s0;
+    ti.bc = 0;
+    if (s0 < 0 || ti.len < 0 || ti.len > p.N || s1 > p.rows_total) {
+      // offsets out of range: skip the tile and report it (only one role does)
+      if (threadIdx.x == 0) atomicCAS(&g_fa_watchdog, 0u, (kRoleArgs << 8) | kSiteSeqlens);
+      ti.len = 0;
+    }
+  } else {
+    ti.row0 = 0;
+    ti.len = p.N;
+    ti.bc = ti.b;
+  }
+  key_range(p, ti.len, ti.q0, ti.lo[0], ti.hi[0]);
+  if (QS == 2)
+    key_range(p, ti.len, ti.q0 + BM, ti.lo[1], ti.hi[1]);
+  else
+    ti.lo[1] = ti.hi[1] = 0;
+  ti.lo_u = ti.lo[0];
+  ti.n_u = ti.hi[0] == 0 ? 0 : max(ti.hi[0], ti.hi[1]) - ti.lo[0];
   return ti;
 }
 
@@ -215,12 +269,14 @@ __host__ __device__ __forceinline__ int ring_k(int j) { return j == 0 ? 0 : 2 * 
 __host__ __device__ __forceinline__ int ring_v(int j, int n) { return j < n - 1 ? 2 * j + 2 : 2 * n - 1; }
 
 // Order in which the Q tiles of a work tile use the shared P buffer: block j
-// of tile 0, then block j of tile 1, then block j + 1 of tile 0, ...  Returns
-// the tile of the use after (s, j), or -1 if (s, j) is the work tile's last.
-__device__ __forceinline__ int next_p_user(int s, int j, const int (&n)[2]) {
-  if (s == 0 && j < n[1]) return 1;
-  if (j + 1 < n[0]) return 0;
-  if (j + 1 < n[1]) return 1;
+// of tile 0 (if in its range), then block j of tile 1 (likewise), then block
+// j + 1, ...  Tile 0's range starts first, so it is every work tile's first
+// user.  Returns the tile of the use after (s, j), or -1 if (s, j) is the
+// work tile's last.
+__device__ __forceinline__ int next_p_user(int s, int j, const TileInfo& ti) {
+  if (s == 0 && in_range(ti, 1, j)) return 1;
+  if (in_range(ti, 0, j + 1)) return 0;
+  if (in_range(ti, 1, j + 1)) return 1;
   return -1;
 }
 
@@ -267,7 +323,7 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
 #pragma unroll
     for (int c = 0; c < C::CHUNKS; ++c)
       tma_load_4d(base + C::SKV_OFF + slot * C::TILE_BYTES + c * C::CHUNK_BYTES, map, full,
-                  c * 64, row0, ti.h, ti.b);
+                  c * 64, ti.row0 + row0, ti.h, ti.bc);
     ++kv_count;
     return true;
   };
@@ -275,9 +331,10 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
     const TileInfo ti = decode_tile<QS>(p, t);
-    // K(0) needs only a ring slot: request it before waiting for the previous
-    // work tile to release the Q buffer, so the two loads overlap.
-    if (!(ok = load_kv(&p.tmap_k, 0, ti))) break;
+    if (ti.n_u == 0) continue;
+    // The first K tile needs only a ring slot: request it before waiting for
+    // the previous work tile to release the Q buffer, so the two loads overlap.
+    if (!(ok = load_kv(&p.tmap_k, ti.lo_u * BN, ti))) break;
     if (q_count > 0) {
       ok = wait_phase(bars + 8 * C::B_Q_EMPTY, (q_count - 1) & 1, abort_flag, p.wait_limit_ns,
                       (kRoleProducer << 8) | kSiteQEmpty);
@@ -289,10 +346,11 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
 #pragma unroll
       for (int c = 0; c < C::CHUNKS; ++c)
         tma_load_4d(base + C::SQ_OFF + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tmap_q,
-                    bars + 8 * C::B_Q_FULL, c * 64, ti.q0 + s * BM, ti.h, ti.b);
+                    bars + 8 * C::B_Q_FULL, c * 64, ti.row0 + ti.q0 + s * BM, ti.h, ti.bc);
     ++q_count;
-    for (int j = 0; ok && j < ti.n_max; ++j) {
-      if (j + 1 < ti.n_max && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
+    for (int jj = 0; ok && jj < ti.n_u; ++jj) {
+      const int j = ti.lo_u + jj;
+      if (jj + 1 < ti.n_u && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
       ok = load_kv(&p.tmap_v, j * BN, ti);
     }
   }
@@ -367,23 +425,25 @@ __device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
     const TileInfo ti = decode_tile<QS>(p, t);
+    if (ti.n_u == 0) continue;
     ok = wait_phase(bars + 8 * C::B_Q_FULL, q_count & 1, abort_flag, lim,
                     (kRoleMma << 8) | kSiteQFull);
     tc_fence_after_sync();
     ++q_count;
     if (!ok) break;
     const int kv0 = kv_count;
-    for (int j = 0; ok && j < ti.n_max; ++j) {
-      const int k_idx = kv0 + ring_k(j);
+    for (int jj = 0; ok && jj < ti.n_u; ++jj) {
+      const int j = ti.lo_u + jj;
+      const int k_idx = kv0 + ring_k(jj);
       if (!(ok = wait_kv(k_idx))) break;
 #pragma unroll 1
       for (int s = 0; s < QS; ++s)
-        if (ok && j < ti.n[s]) ok = issue_s(s, k_idx % KVS);
+        if (ok && in_range(ti, s, j)) ok = issue_s(s, k_idx % KVS);
       if (!ok) break;
       tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
-      if (j + 1 == ti.n_max) tc_commit(bars + 8 * C::B_Q_EMPTY);
+      if (jj + 1 == ti.n_u) tc_commit(bars + 8 * C::B_Q_EMPTY);
     }
-    kv_count = kv0 + 2 * ti.n_max;
+    kv_count = kv0 + 2 * ti.n_u;
   }
   if (!ok) {
     // Wait for every MMA this thread issued before TMEM is released.
@@ -441,25 +501,27 @@ __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
     const TileInfo ti = decode_tile<QS>(p, t);
+    if (ti.n_u == 0) continue;
     const int kv0 = kv_count;
-    for (int j = 0; ok && j < ti.n_max; ++j) {
-      const int v_idx = kv0 + ring_v(j, ti.n_max);
+    for (int jj = 0; ok && jj < ti.n_u; ++jj) {
+      const int j = ti.lo_u + jj;
+      const int v_idx = kv0 + ring_v(jj, ti.n_u);
       ok = wait_phase(bars + 8 * (C::B_KV_FULL + v_idx % KVS), (v_idx / KVS) & 1, abort_flag, lim,
                       (kRoleMma << 8) | kSiteKvFull);
       tc_fence_after_sync();
 #pragma unroll 1
       for (int s = 0; s < QS; ++s) {
-        if (!ok || j >= ti.n[s]) continue;
+        if (!ok || !in_range(ti, s, j)) continue;
         // the next work tile starts with tile 0
-        const int nxt = next_p_user(s, j, ti.n);
-        ok = issue_pv(s, v_idx % KVS, j > 0, nxt < 0 ? 0 : nxt);
+        const int nxt = next_p_user(s, j, ti);
+        ok = issue_pv(s, v_idx % KVS, j > ti.lo[s], nxt < 0 ? 0 : nxt);
         if (!ok) break;
-        if (j == ti.n[s] - 1) tc_commit(bars + 8 * (C::B_O_FINAL + s));
+        if (j == ti.hi[s] - 1) tc_commit(bars + 8 * (C::B_O_FINAL + s));
       }
       if (!ok) break;
       tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
     }
-    kv_count = kv0 + 2 * ti.n_max;
+    kv_count = kv0 + 2 * ti.n_u;
   }
   if (!ok) {
     volatile int no_abort = 0;
@@ -546,7 +608,9 @@ __device__ __forceinline__ void softmax_chunk(const float* sv, float sl2, float 
   }
 }
 
-template <int HD, int QS, int KVS, bool BF16>
+// ALIBI: the scaled score of key j gets -slope[h] * |i - j| (in the log2
+// domain, -slope[h] * log2(e) * |i - j|) before the row max is taken.
+template <int HD, int QS, int KVS, bool BF16, bool ALIBI>
 __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
                              volatile int* abort_flag) {
   using C = FwdCfg<HD, QS, KVS, BF16>;
@@ -589,16 +653,18 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
     const TileInfo ti = decode_tile<QS>(p, t);
-    const int n = ti.n[s];
-    if (n == 0) continue;
-    const int row = ti.q0 + s * BM + r;
-    // keys visible from this row: [0, limit)
-    const int limit = p.causal ? min(row + 1, p.N) : p.N;
-    // first key block that needs the mask
-    const int first_masked = p.causal ? ((ti.q0 + s * BM) / BN) : (p.N / BN);
+    const int lo = ti.lo[s], hi = ti.hi[s];
+    if (lo == hi) continue;
+    const int r_first = ti.q0 + s * BM, r_last = r_first + BM - 1;
+    const int row = r_first + r;  // relative to the sequence
+    // keys visible from this row: [vis_lo, vis_hi)
+    const int vis_lo = p.window_left < 0 ? 0 : row - p.window_left;
+    const int vis_hi = p.window_right < 0 ? ti.len : min(ti.len, row + p.window_right + 1);
+    float nslope2 = 0.f;  // -slope * log2(e)
+    if constexpr (ALIBI) nslope2 = -__ldg(p.alibi_slopes + ti.h) * 1.4426950408889634f;
     float m_ref = -INFINITY, l = 0.f;
 
-    for (int j = 0; j < n; ++j) {
+    for (int j = lo; j < hi; ++j) {
       bool ok = wait_phase(bars + 8 * (C::B_S_FULL + s), s_par, abort_flag, lim,
                            (kRoleSoftmax << 8) | kSiteSFull);
       s_par ^= 1u;
@@ -610,14 +676,30 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       float sv[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c]);
-      const bool need_mask = j >= first_masked;
+      // Blocks where some key is invisible to some row of the tile: the ragged
+      // tail, the causal diagonal, the edges of a local window.
+      const bool need_mask =
+          (j * BN + BN > ti.len) ||
+          (p.window_left >= 0 && j * BN < r_last - p.window_left) ||
+          (p.window_right >= 0 && j * BN + BN - 1 > r_first + p.window_right);
+      const int kbase = j * BN + 64 * hf;  // key of this thread's first column
       if (need_mask) {
-        const int lim_local = limit - j * BN - 64 * hf;
+        const int lo_c = vis_lo - kbase, hi_c = vis_hi - kbase;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) sv[c] = (c < lim_local) ? sv[c] : -INFINITY;
+        for (int c = 0; c < 64; ++c) sv[c] = (c >= lo_c && c < hi_c) ? sv[c] : -INFINITY;
       }
-      // row max over both halves of the row
-      const float m_half = row_max64(sv) * sl2;
+      float m_half;
+      if constexpr (ALIBI) {
+        // log2-domain biased scores; the max is taken over them
+        const float dist0 = static_cast<float>(row - kbase);
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          sv[c] = fmaf(sv[c], sl2, nslope2 * fabsf(dist0 - static_cast<float>(c)));
+        m_half = row_max64(sv);
+      } else {
+        // row max over both halves of the row
+        m_half = row_max64(sv) * sl2;
+      }
       x_mine[r] = m_half;
       if (!group_meet()) return;
       const float m_blk = fmaxf(m_half, x_other[r]);
@@ -631,11 +713,15 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       // Lazy reference: keep m_ref unless the block max exceeds it by more
       // than 2^8; the first block always sets it.  Both groups of the tile
       // take the same decision from the same values.
-      const bool rescale = (j > 0) && (m_blk > m_ref + kLazyRescaleLog2);
-      const float m_new = (j == 0 || rescale) ? m_blk : m_ref;
-      const float alpha = (j == 0) ? 0.f : ex2(m_ref - m_new);  // 1 when m_ref is kept
+      // A row with no visible key so far (m_ref = -inf: only possible at the
+      // edges of a local window) has l = 0 and O = 0, so its alpha is 0.
+      const bool rescale = (j > lo) && (m_blk > m_ref + kLazyRescaleLog2);
+      const float m_new = (j == lo || rescale) ? m_blk : m_ref;
+      const float alpha =
+          (j == lo || m_ref == -INFINITY) ? 0.f : ex2(m_ref - m_new);  // 1 when m_ref is kept
       m_ref = m_new;
       const float neg_ref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      const float sl2e = ALIBI ? 1.f : sl2;  // the ALiBi path holds scaled scores already
 
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
@@ -643,9 +729,9 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         if (need_mask)
-          softmax_chunk<BF16, 0>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
+          softmax_chunk<BF16, 0>(sv + 32 * c, sl2e, neg_ref, pk + 16 * c, acc);
         else
-          softmax_chunk<BF16, poly_pairs_per8<HD>()>(sv + 32 * c, sl2, neg_ref, pk + 16 * c, acc);
+          softmax_chunk<BF16, poly_pairs_per8<HD>()>(sv + 32 * c, sl2e, neg_ref, pk + 16 * c, acc);
       }
       // This group's half of the P buffer is this tile's turn: the previous
       // user's K-steps that read it have run.
@@ -706,8 +792,10 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const float l_row = l + x_other[r];
     if (!group_meet()) return;  // both have read before the slots are reused
     const float inv_l = 1.f / l_row;
-    T* orow = reinterpret_cast<T*>(p.o) + ti.b * p.o_stride_b + ti.h * p.o_stride_h +
-              static_cast<long long>(row) * p.o_stride_n + HD2 * hf;
+    const long long trow = static_cast<long long>(ti.row0) + row;  // tensor row
+    const bool store = row < ti.len && trow < p.rows_total;
+    T* orow = reinterpret_cast<T*>(p.o) + ti.bc * p.o_stride_b + ti.h * p.o_stride_h +
+              trow * p.o_stride_n + HD2 * hf;
 #pragma unroll 1
     for (int c = 0; c < HD2; c += 32) {
       uint32_t ov[32];
@@ -717,14 +805,14 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
 #pragma unroll
       for (int i = 0; i < 16; ++i)
         wp[i] = pack2<BF16>(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
-      if (row < p.N) {
+      if (store) {
         uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[i] = w[i];
       }
     }
-    if (hf == 0 && p.lse != nullptr && row < p.N)
-      p.lse[(static_cast<long long>(ti.b) * p.H + ti.h) * p.N + row] =
+    if (hf == 0 && p.lse != nullptr && store)
+      p.lse[ti.bc * p.lse_stride_b + ti.h * p.lse_stride_h + trow] =
           (m_ref + log2f(l_row)) * 0.69314718055994530942f;
     // The next tile's first P V overwrites O only after this group's next
     // P arrival, which comes after these loads completed.
@@ -732,7 +820,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   }
 }
 
-template <int HD, int QS, int KVS, bool BF16>
+template <int HD, int QS, int KVS, bool BF16, bool ALIBI>
 __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<HD, QS, KVS, BF16>;
@@ -796,7 +884,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
   }
 
   if (warp < C::SOFTMAX_WARPS) {
-    softmax_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
+    softmax_role<HD, QS, KVS, BF16, ALIBI>(p, base, tmem, abort_flag);
   } else if (warp == C::PRODUCER_WARP) {
     if (lane == 0) producer_role<HD, QS, KVS, BF16>(p, base, abort_flag);
   } else if (warp == C::MMA_S_WARP) {

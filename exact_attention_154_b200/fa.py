@@ -23,12 +23,18 @@ _lib = None
 FA_OK = 0
 FA_ERR_ARG, FA_ERR_ALIGN, FA_ERR_HEADDIM, FA_ERR_DTYPE = -1, -2, -3, -4
 FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_DEVICE = -5, -6, -7, -8
+FA_ERR_SEQLENS = -9
 
 #: every function the C header declares, with (restype, argtypes)
 _VP, _FP, _I, _F = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_fwd_qkvpacked": (_I, [_VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _F, _I, _VP]),
+    "fa_fwd_ext": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I, _I, _FP, _I, _VP]),
+    "fa_fwd_qkvpacked_ext": (_I, [_VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _F, _I, _I, _FP, _I,
+                                  _VP]),
+    "fa_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _I, _FP,
+                           _I, _VP]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I,
                     _VP]),
     "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I,
@@ -114,13 +120,34 @@ def _check_tensor(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _window(window) -> tuple[int, int]:
+    left, right = (int(window[0]), int(window[1]))
+    return left, right
+
+
+def _slopes(alibi_slopes, H: int, dev: torch.device):
+    """The ``[H]`` fp32 slope tensor on ``dev`` (or None) and its pointer."""
+    if alibi_slopes is None:
+        return None, None
+    if not isinstance(alibi_slopes, torch.Tensor):
+        alibi_slopes = torch.as_tensor(alibi_slopes, dtype=torch.float32)
+    if alibi_slopes.shape != (H,) or alibi_slopes.dtype != torch.float32:
+        raise ValueError("alibi_slopes must be a float32 tensor of shape [H]")
+    alibi_slopes = alibi_slopes.to(dev).contiguous()
+    return alibi_slopes, alibi_slopes.data_ptr()
+
+
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None = None,
         causal: bool = False, out: torch.Tensor | None = None,
-        lse: torch.Tensor | None = None, return_lse: bool = True):
+        lse: torch.Tensor | None = None, return_lse: bool = True,
+        window_size=(-1, -1), alibi_slopes=None):
     """Attention forward on ``[B, H, N, d]`` tensors (``[B, N, d]`` is taken as H=1).
 
     Returns ``(O, LSE)`` (``LSE`` is ``[B, H, N]`` fp32, or None when
     ``return_lse`` is False).  ``scale=None`` means ``1/sqrt(d)``.
+    ``window_size=(left, right)``: key j visible from query i iff
+    ``i - left <= j <= i + right`` (-1: unbounded).  ``alibi_slopes``: ``[H]``
+    fp32; the scaled score gets ``-slope[h] * |i - j|``.
     """
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_tensor(t, name)
@@ -150,19 +177,24 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: float | None =
         lse = None
     dev = same_device([("q", q), ("k", k), ("v", v), ("out", out)] +
                       ([("lse", lse)] if lse is not None else []))
+    left, right = _window(window_size)
+    slopes, slopes_ptr = _slopes(alibi_slopes, H, dev)
     with _on(dev):
-        rc = load().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse_ptr,
-                           B, H, N, d, 0.0 if scale is None else float(scale),
-                           int(bool(causal)), _DT[q.dtype], _stream_ptr(q))
+        rc = load().fa_fwd_ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse_ptr, B, H, N, d, 0.0 if scale is None else float(scale),
+                               int(bool(causal)), left, right, slopes_ptr, _DT[q.dtype],
+                               _stream_ptr(q))
     if rc != FA_OK:
-        raise FaError(rc, "fa_fwd")
+        raise FaError(rc, "fa_fwd_ext")
     return out, lse
 
 
 def fwd_qkvpacked(qkv: torch.Tensor, dropout_p: float = 0.0, softmax_scale: float | None = None,
                   causal: bool = False, out: torch.Tensor | None = None,
-                  return_lse: bool = True):
-    """Packed forward: ``qkv`` is ``[B, N, 3, H, d]``; returns ``(O [B, N, H, d], LSE [B, H, N])``."""
+                  return_lse: bool = True, window_size=(-1, -1), alibi_slopes=None):
+    """Packed forward: ``qkv`` is ``[B, N, 3, H, d]``; returns ``(O [B, N, H, d], LSE [B, H, N])``.
+
+    ``window_size`` and ``alibi_slopes`` as :func:`fwd`."""
     _check_tensor(qkv, "qkv")
     if qkv.dim() != 5 or qkv.shape[2] != 3:
         raise ValueError("qkv must be [B, N, 3, H, d]")
@@ -175,13 +207,47 @@ def fwd_qkvpacked(qkv: torch.Tensor, dropout_p: float = 0.0, softmax_scale: floa
         raise ValueError("out must be [B, N, H, d] in qkv's dtype")
     lse = torch.empty((B, H, N), device=qkv.device, dtype=torch.float32) if return_lse else None
     dev = same_device([("qkv", qkv), ("out", out)])
+    left, right = _window(window_size)
+    slopes, slopes_ptr = _slopes(alibi_slopes, H, dev)
     with _on(dev):
-        rc = load().fa_fwd_qkvpacked(
+        rc = load().fa_fwd_qkvpacked_ext(
             qkv.data_ptr(), out.data_ptr(), None if lse is None else lse.data_ptr(), B, N, H, d,
             0.0 if softmax_scale is None else float(softmax_scale), int(bool(causal)),
-            float(dropout_p), _DT[qkv.dtype], _stream_ptr(qkv))
+            float(dropout_p), left, right, slopes_ptr, _DT[qkv.dtype], _stream_ptr(qkv))
     if rc != FA_OK:
-        raise FaError(rc, "fa_fwd_qkvpacked")
+        raise FaError(rc, "fa_fwd_qkvpacked_ext")
+    return out, lse
+
+
+def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+               max_seqlen: int, scale: float | None = None, causal: bool = False,
+               window_size=(-1, -1), alibi_slopes=None, return_lse: bool = True):
+    """Forward over sequences packed back to back: ``q, k, v`` are
+    ``[total, H, d]``, sequence b holds rows ``cu_seqlens[b] .. cu_seqlens[b+1]-1``
+    (``cu_seqlens``: int32 ``[batch + 1]`` on the same device).  Returns
+    ``(O [total, H, d], LSE [H, total])``.  Masks as :func:`fwd`, per sequence."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(t, name)
+    if not (q.shape == k.shape == v.shape) or q.dim() != 3 or len({q.dtype, k.dtype, v.dtype}) != 1:
+        raise ValueError("q, k, v must share one [total, H, d] shape and dtype")
+    if (not isinstance(cu_seqlens, torch.Tensor) or cu_seqlens.dtype != torch.int32
+            or cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2 or not cu_seqlens.is_contiguous()):
+        raise ValueError("cu_seqlens must be a contiguous int32 tensor of batch + 1 offsets")
+    total, H, d = q.shape
+    batch = cu_seqlens.numel() - 1
+    dev = same_device([("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens)])
+    out = torch.empty_like(q)
+    lse = torch.empty((H, total), device=dev, dtype=torch.float32) if return_lse else None
+    left, right = _window(window_size)
+    slopes, slopes_ptr = _slopes(alibi_slopes, H, dev)
+    with _on(dev):
+        rc = load().fa_fwd_varlen(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+            None if lse is None else lse.data_ptr(), cu_seqlens.data_ptr(), batch,
+            int(max_seqlen), total, H, d, 0.0 if scale is None else float(scale),
+            int(bool(causal)), left, right, slopes_ptr, _DT[q.dtype], _stream_ptr(q))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_varlen")
     return out, lse
 
 

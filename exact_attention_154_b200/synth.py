@@ -35,8 +35,12 @@ DTYPE_NAME = {FP16: "f16", BF16: "bf16"}
 class Workload:
     """One attention forward problem.
 
-    ``layout`` is ``"bhnd"`` (separate q, k, v of shape [B, H, N, d]) or
-    ``"packed"`` (one qkv of shape [B, N, 3, H, d]).
+    ``layout`` is ``"bhnd"`` (separate q, k, v of shape [B, H, N, d]),
+    ``"packed"`` (one qkv of shape [B, N, 3, H, d]) or ``"varlen"``
+    (``lengths`` sequences packed back to back as [total, H, d]; B is the
+    number of sequences and N the longest length).  ``window`` is the local
+    window (left, right), -1 = unbounded; ``alibi`` adds the usual per-head
+    ALiBi slopes (:func:`alibi_slopes`).
     """
     name: str
     B: int
@@ -50,21 +54,53 @@ class Workload:
     sigma_qk: float = 1.0
     sigma_v: float = 1.0
     extra: dict = field(default_factory=dict, compare=False)
+    window: tuple = (-1, -1)
+    alibi: bool = False
+    lengths: tuple = ()
 
     @property
     def scale(self) -> float:
         return 1.0 / math.sqrt(self.d)
 
     @property
+    def masked(self) -> bool:
+        return self.window != (-1, -1) or self.alibi or self.layout == "varlen"
+
+    @property
     def flops(self) -> float:
-        """4*B*H*N^2*d, halved for the causal mask."""
-        f = 4.0 * self.B * self.H * self.N * self.N * self.d
-        return f / 2 if self.causal else f
+        """4*B*H*N^2*d, halved for the causal mask; with a local window or
+        variable lengths, 4*d*H per (query, visible key) pair, counted exactly."""
+        if not self.masked or (self.window == (-1, -1) and self.layout != "varlen"):
+            f = 4.0 * self.B * self.H * self.N * self.N * self.d
+            return f / 2 if self.causal else f
+        lengths = self.lengths if self.layout == "varlen" else (self.N,) * self.B
+        return 4.0 * self.d * self.H * sum(visible_pairs(n, self.causal, self.window)
+                                           for n in lengths)
 
     def describe(self) -> dict:
-        return {"workload": self.name, "B": self.B, "H": self.H, "N": self.N,
-                "d": self.d, "dtype": DTYPE_NAME[self.dtype],
-                "causal": self.causal, "layout": self.layout, "seed": self.seed}
+        out = {"workload": self.name, "B": self.B, "H": self.H, "N": self.N,
+               "d": self.d, "dtype": DTYPE_NAME[self.dtype],
+               "causal": self.causal, "layout": self.layout, "seed": self.seed}
+        if self.window != (-1, -1):
+            out["window"] = list(self.window)
+        if self.alibi:
+            out["alibi"] = "2^(-8(h+1)/H)"
+        if self.layout == "varlen":
+            out["total_tokens"] = int(sum(self.lengths))
+        return out
+
+
+def visible_pairs(n: int, causal: bool, window=(-1, -1)) -> int:
+    """Number of (query, key) pairs with key j visible from query i in a
+    sequence of n tokens: i - left <= j <= i + right (-1 unbounded), j <= i
+    when causal."""
+    left, right = window
+    if causal:
+        right = 0
+    i = np.arange(n, dtype=np.int64)
+    lo = np.zeros(n, np.int64) if left < 0 else np.maximum(i - left, 0)
+    hi = np.full(n, n - 1, np.int64) if right < 0 else np.minimum(i + right, n - 1)
+    return int((hi - lo + 1).sum())
 
 
 def single_head_n256() -> Workload:
@@ -99,6 +135,40 @@ def headdim256_causal() -> Workload:
                     1, 8, 8192, 256, BF16, True, 50, sigma_qk=3.0)
 
 
+def window_causal_n4096() -> Workload:
+    """The N = 4096 sweep shape with a causal sliding window of 256 keys."""
+    return Workload("sliding-window causal fwd B=4,H=16,N=4096,d=128 bf16, window (256, 0)",
+                    4, 16, 4096, 128, BF16, True, 60, window=(256, 0))
+
+
+def alibi_causal_n4096() -> Workload:
+    """The N = 4096 sweep shape, causal, with per-head ALiBi slopes."""
+    return Workload("ALiBi causal fwd B=4,H=16,N=4096,d=128 bf16", 4, 16, 4096, 128, BF16,
+                    True, 61, alibi=True)
+
+
+def varlen_lengths(seed: int, total: int, lo: int, hi: int) -> tuple:
+    """Seeded sequence lengths, uniform in [lo, hi], until ``total`` tokens
+    (the last one trimmed)."""
+    rng = np.random.default_rng(seed)
+    out, acc = [], 0
+    while acc < total:
+        n = int(min(rng.integers(lo, hi + 1), total - acc))
+        out.append(n)
+        acc += n
+    return tuple(out)
+
+
+def varlen_mix_causal() -> Workload:
+    """Sequences of 128..8192 tokens (seeded, uniform) packed to 65536 tokens,
+    H=16, d=128, bf16, causal: a dynamic-length batch of the size of the
+    N = 4096 sweep point times four."""
+    lengths = varlen_lengths(62, 65536, 128, 8192)
+    return Workload(f"varlen causal fwd {len(lengths)} sequences of 128..8192 tokens "
+                    f"(65536 total), H=16, d=128 bf16", len(lengths), 16, max(lengths), 128,
+                    BF16, True, 62, layout="varlen", lengths=lengths)
+
+
 def all_workloads() -> list[Workload]:
     w = [single_head_n256(), packed_qkv_b2_n256_h12(), many_heads_causal_n2048()]
     for n in SWEEP_N:
@@ -112,10 +182,14 @@ def make_inputs(w: Workload):
     """CPU tensors in the compute dtype.
 
     ``bhnd`` -> ``(q, k, v)`` each [B, H, N, d]; ``packed`` -> ``(qkv,)`` of
-    shape [B, N, 3, H, d] (index 0/1/2 of axis 2 = q/k/v).
+    shape [B, N, 3, H, d] (index 0/1/2 of axis 2 = q/k/v); ``varlen`` ->
+    ``(q, k, v, cu_seqlens)`` with q, k, v [total, H, d].
     """
     g = torch.Generator().manual_seed(w.seed)
     dt = TORCH_DTYPE[w.dtype]
+    if w.layout == "varlen":
+        q, k, v, cu = packed_lengths(w.lengths, w.H, w.d, w.dtype, w.seed, w.sigma_qk, w.sigma_v)
+        return q, k, v, cu
     if w.layout == "packed":
         qkv = torch.randn((w.B, w.N, 3, w.H, w.d), generator=g, dtype=torch.float32)
         qkv[:, :, 0:2] *= w.sigma_qk
@@ -144,6 +218,27 @@ def sample_rows(N: int, seed: int, count: int = 512) -> np.ndarray:
     rng = np.random.default_rng(seed + 1000)
     pick = rng.choice(N, size=count, replace=False)
     return np.array(sorted(must.union(int(x) for x in pick)), dtype=np.int32)
+
+
+def alibi_slopes(H: int) -> torch.Tensor:
+    """The usual ALiBi slopes for H heads, 2^(-8 (h + 1) / H), as an fp32 [H]
+    tensor (an input like q, k, v; the pages give the keyword, not values)."""
+    return torch.tensor([2.0 ** (-8.0 * (h + 1) / H) for h in range(H)], dtype=torch.float32)
+
+
+def packed_lengths(lengths, H, d, dtype, seed, sigma_qk=1.0, sigma_v=1.0, extra_rows=0):
+    """Sequences of the given lengths packed back to back: ``(q, k, v)`` each
+    ``[total, H, d]`` (same recipe as :func:`make_inputs`), plus the int32
+    offsets ``cu_seqlens`` ``[len(lengths) + 1]``.  ``extra_rows`` trailing rows
+    belong to no sequence."""
+    total = int(sum(lengths)) + extra_rows
+    g = torch.Generator().manual_seed(seed)
+    dt = TORCH_DTYPE[dtype]
+    q = torch.randn((total, H, d), generator=g, dtype=torch.float32) * sigma_qk
+    k = torch.randn((total, H, d), generator=g, dtype=torch.float32) * sigma_qk
+    v = torch.randn((total, H, d), generator=g, dtype=torch.float32) * sigma_v
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+    return q.to(dt), k.to(dt), v.to(dt), cu
 
 
 def random_inputs(B, H, N, d, dtype, seed, sigma_qk=1.0, sigma_v=1.0):

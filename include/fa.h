@@ -1,7 +1,8 @@
 /*
  * fa.h -- C ABI of the B200 (sm_100a) exact attention library (libfa_sm100.so):
- * the forward (fa_fwd, fa_fwd_qkvpacked) and its gradient (fa_bwd,
- * fa_bwd_noalloc).
+ * the forward (fa_fwd, fa_fwd_qkvpacked; with a local window and ALiBi
+ * fa_fwd_ext, fa_fwd_qkvpacked_ext; over variable-length sequences
+ * fa_fwd_varlen) and its gradient (fa_bwd, fa_bwd_noalloc).
  *
  * Operation.  For every batch b, head h and query row i:
  *
@@ -52,7 +53,8 @@ enum fa_status {
   FA_ERR_UNSUPPORTED = -5, /* dropout_p != 0 */
   FA_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
   FA_ERR_TIMEOUT = -7,     /* a kernel gave up on a bounded wait */
-  FA_ERR_DEVICE = -8       /* the current device is not sm_100 (B200 class) */
+  FA_ERR_DEVICE = -8,      /* the current device is not sm_100 (B200 class) */
+  FA_ERR_SEQLENS = -9      /* (fa_device_status) a kernel met cu_seqlens out of range */
 };
 
 enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1 };
@@ -90,6 +92,71 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
  */
 int fa_fwd_qkvpacked(const void *qkv, void *o, float *lse, int B, int N, int H, int d, float scale,
                      int causal, float dropout_p, int dtype, struct CUstream_st *stream);
+
+/*
+ * fa_fwd with the two masks the packed call's keyword list names besides
+ * `causal`: a local window (window_size) and an ALiBi bias (alibi_slopes);
+ * section 10.1 (and 5.2) of "Windows下RTX 3090编译Flash Attention 2.8.3全指南"
+ * (intelliparadigm.com).  The page lists both keywords without defining them;
+ * the reading taken here:
+ *
+ *   window_left, window_right : key j is visible from query i iff
+ *       i - window_left <= j <= i + window_right, intersected with the causal
+ *       mask when causal != 0; -1 leaves that side unbounded (window_size =
+ *       (-1, -1) is the plain forward).  Values below -1 give FA_ERR_ARG.
+ *       Every row sees at least its own key.
+ *   alibi_slopes : device pointer to H fp32 slopes, or NULL.  The scaled score
+ *       of key j in head h becomes scale * q_i . k_j - alibi_slopes[h] * |i - j|
+ *       (the softmax, O and LSE are taken over these biased scores).  Slopes
+ *       must be finite.  4-byte alignment required.
+ *
+ * Other arguments, layouts, results and errors as fa_fwd; fa_fwd is this call
+ * with (-1, -1, NULL).  Key blocks that lie wholly outside every row's window
+ * are neither loaded nor multiplied.
+ */
+int fa_fwd_ext(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+               int N, int d, float scale, int causal, int window_left, int window_right,
+               const float *alibi_slopes, int dtype, struct CUstream_st *stream);
+
+/*
+ * fa_fwd_qkvpacked with the local window and ALiBi bias of fa_fwd_ext: the
+ * full keyword list of flash_attn_qkvpacked_func in section 10.1 of the
+ * intelliparadigm.com guide except `deterministic` (this forward is always
+ * deterministic: one fixed reduction order per output element).
+ */
+int fa_fwd_qkvpacked_ext(const void *qkv, void *o, float *lse, int B, int N, int H, int d,
+                         float scale, int causal, float dropout_p, int window_left,
+                         int window_right, const float *alibi_slopes, int dtype,
+                         struct CUstream_st *stream);
+
+/*
+ * Forward over a batch of sequences of different lengths packed back to back
+ * (the dynamic sequence lengths of item 3, "动态形状优化", of
+ * "flash-attention与TensorRT 10集成", blog.gitcode.com): sequence b holds the
+ * tokens cu_seqlens[b] .. cu_seqlens[b+1]-1, attends only to itself, and
+ * query and key lengths are equal (self-attention).
+ *
+ *   q, k, v    : [total, H, d] contiguous, element type `dtype`
+ *   o          : [total, H, d] contiguous (written)
+ *   lse        : [H, total] fp32 (written), or NULL
+ *   cu_seqlens : device pointer to batch + 1 int32 offsets, nondecreasing,
+ *                cu_seqlens[0] = 0, cu_seqlens[batch] <= total
+ *   batch      : number of sequences (>= 1)
+ *   max_seqlen : >= every sequence length (host value; sizes the grid)
+ *   total      : rows of q, k, v, o (>= 1)
+ *   causal, window_left, window_right, alibi_slopes : per sequence, positions
+ *                counted from the sequence's first token; as fa_fwd_ext
+ *   other arguments as fa_fwd.
+ *
+ * The offsets are read on the device only.  A sequence whose offsets are out
+ * of range (negative, decreasing, longer than max_seqlen, or past total) is
+ * skipped -- its rows of o and lse are not written -- and fa_device_status()
+ * then returns FA_ERR_SEQLENS.  All rows of q, k, v must hold finite values.
+ */
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens, int batch, int max_seqlen, int total, int H, int d,
+                  float scale, int causal, int window_left, int window_right,
+                  const float *alibi_slopes, int dtype, struct CUstream_st *stream);
 
 /*
  * Gradient of fa_fwd: dQ, dK, dV for an upstream gradient dO of O.  The score
@@ -139,8 +206,9 @@ const char *fa_strerror(int status);
 /*
  * Reads (and, if clear != 0, resets) the current device's watchdog word.
  * Synchronises the current device first.  Returns FA_OK, FA_ERR_TIMEOUT when a
- * kernel gave up on a bounded wait (`*detail`, if not NULL, receives the
- * (role << 8) | site code), or FA_ERR_CUDA.
+ * kernel gave up on a bounded wait, FA_ERR_SEQLENS when fa_fwd_varlen met
+ * offsets out of range (`*detail`, if not NULL, receives the (role << 8) | site
+ * code), or FA_ERR_CUDA.
  */
 int fa_device_status(int clear, unsigned int *detail);
 

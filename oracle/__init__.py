@@ -20,13 +20,17 @@ Three independent implementations live here:
 * :func:`attention_masked` -- the definition with a local window and an
   ALiBi bias (the two masks the packed call names), pinned in
   ``tests/test_oracle_mask_pins.py``.
+* :func:`attention_varlen` -- sequences of different lengths packed back to
+  back (``[total, H, d]`` with ``cu_seqlens`` offsets): the definition applied
+  to each sequence on its own, pinned in ``tests/test_oracle_varlen_pins.py``.
 * :func:`attention_bwd` -- the gradient of the plain definition with respect
   to q, k, v (chain rule written out in ``fa_oracle.c``), pinned in
   ``tests/test_oracle_bwd_pins.py`` by central finite differences of
   :func:`attention`, closed forms and invariants.
 
 Parity status: every function here is pinned by tests in
-``tests/test_oracle_pins.py``, ``tests/test_oracle_mask_pins.py`` and
+``tests/test_oracle_pins.py``, ``tests/test_oracle_mask_pins.py``,
+``tests/test_oracle_varlen_pins.py`` and
 ``tests/test_oracle_bwd_pins.py`` (closed
 forms, invariants, brute force, finite differences and the
 recurrence-equals-definition check); none is "parity unpinned".
@@ -195,6 +199,40 @@ def attention_masked(q, k, v, scale: float | None = None, causal: bool = False,
     if rc != 0:
         raise ValueError(f"oracle_attention_fwd_masked failed ({rc})")
     return o.reshape(lead + (nr, d)), lse.reshape(lead + (nr,))
+
+
+def attention_varlen(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = False,
+                     window=(-1, -1), alibi_slopes=None):
+    """Attention over sequences packed back to back, in fp64.
+
+    ``q, k, v``: ``[total, H, d]``; sequence b is rows ``cu_seqlens[b]`` to
+    ``cu_seqlens[b+1] - 1`` and attends only to itself, with positions counted
+    from its first row (the dynamic sequence lengths of item 3, "动态形状优化",
+    of "flash-attention与TensorRT 10集成", blog.gitcode.com, read as independent
+    self-attention problems of their own lengths).  Each sequence is handed to
+    :func:`attention_masked` as one ``[1, H, L, d]`` problem.
+
+    Returns ``(O [total, H, d], LSE [H, total])``; rows outside every sequence
+    are NaN.
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    if not (q.shape == k.shape == v.shape) or q.ndim != 3:
+        raise ValueError("q, k, v must share one [total, H, d] shape")
+    cu = [int(x) for x in np.asarray(cu_seqlens).reshape(-1)]
+    total, H, d = q.shape
+    if len(cu) < 2 or cu[0] < 0 or cu[-1] > total or any(b < a for a, b in zip(cu, cu[1:])):
+        raise ValueError("cu_seqlens must be nondecreasing offsets within [0, total]")
+    O = np.full((total, H, d), np.nan)
+    LSE = np.full((H, total), np.nan)
+    for s0, s1 in zip(cu, cu[1:]):
+        if s1 == s0:
+            continue
+        seq = [np.ascontiguousarray(t[s0:s1].transpose(1, 0, 2))[None] for t in (q, k, v)]
+        o, lse = attention_masked(*seq, scale=scale, causal=causal, window=window,
+                                  alibi_slopes=alibi_slopes)
+        O[s0:s1] = o[0].transpose(1, 0, 2)
+        LSE[:, s0:s1] = lse[0]
+    return O, LSE
 
 
 def attention_bwd(q, k, v, dout, scale: float | None = None, causal: bool = False):

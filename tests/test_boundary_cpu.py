@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_strerror(lib):
     assert fa.version() >= 10000
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         assert fa.strerror(code) != "unknown status"
     assert fa.strerror(-99) == "unknown status"
 
@@ -126,3 +126,47 @@ def test_bwd_argument_errors(lib):
     assert call(o=P + 2) == fa.FA_ERR_ALIGN
     assert call(lse=P + 2) == fa.FA_ERR_ALIGN
     assert call(ws=P + 1) == fa.FA_ERR_ALIGN
+
+
+def test_ext_argument_errors(lib):
+    def call(q=P, left=-1, right=-1, slopes=None, N=256, causal=0, lse=None):
+        return lib.fa_fwd_ext(q, P, P, P, lse, 1, 2, N, 64, 0.0, causal, left, right, slopes, 1,
+                              None)
+    assert call(q=None) == fa.FA_ERR_ARG
+    assert call(left=-2) == fa.FA_ERR_ARG
+    assert call(right=-3, causal=1) == fa.FA_ERR_ARG
+    assert call(slopes=P + 2) == fa.FA_ERR_ALIGN
+    assert call(q=P + 4, left=5) == fa.FA_ERR_ALIGN
+
+    def packed(qkv=P, dropout=0.0, left=-1, right=-1, slopes=None):
+        return lib.fa_fwd_qkvpacked_ext(qkv, P, None, 2, 256, 4, 64, 0.0, 0, dropout, left, right,
+                                        slopes, 0, None)
+    assert packed(qkv=None) == fa.FA_ERR_ARG
+    assert packed(dropout=0.5) == fa.FA_ERR_UNSUPPORTED
+    assert packed(left=-7) == fa.FA_ERR_ARG
+    assert packed(slopes=P + 1) == fa.FA_ERR_ALIGN
+
+
+def test_varlen_argument_errors(lib):
+    def call(q=P, cu=P, batch=2, max_seqlen=128, total=200, H=2, d=64, dtype=0, slopes=None,
+             left=-1):
+        return lib.fa_fwd_varlen(q, P, P, P, None, cu, batch, max_seqlen, total, H, d, 0.0, 0, left,
+                                 -1, slopes, dtype, None)
+    assert call(cu=None) == fa.FA_ERR_ARG
+    assert call(q=None) == fa.FA_ERR_ARG
+    assert call(batch=0) == fa.FA_ERR_ARG
+    assert call(max_seqlen=0) == fa.FA_ERR_ARG
+    assert call(total=0) == fa.FA_ERR_ARG
+    assert call(d=48) == fa.FA_ERR_HEADDIM
+    assert call(dtype=5) == fa.FA_ERR_DTYPE
+    assert call(left=-4) == fa.FA_ERR_ARG
+    assert call(cu=P + 2) == fa.FA_ERR_ALIGN
+    assert call(slopes=P + 2) == fa.FA_ERR_ALIGN
+    assert call(q=P + 8) == fa.FA_ERR_ALIGN
+
+
+def test_python_varlen_rejects_bad_offsets_tensor():
+    import torch
+    x = torch.zeros(8, 2, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        fa.fwd_varlen(x, x, x, torch.tensor([0, 8], dtype=torch.int64), 8)
