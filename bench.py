@@ -57,6 +57,8 @@ def workloads_by_key():
         "window256-causal-n4096": synth.window_causal_n4096(),
         "alibi-causal-n4096": synth.alibi_causal_n4096(),
         "varlen-mix-causal": synth.varlen_mix_causal(),
+        "fp8-n4096": synth.fp8_sweep_n4096(False),
+        "fp8-n4096-causal": synth.fp8_sweep_n4096(True),
     }
     for n in synth.SWEEP_N:
         table[f"sweep-n{n}"] = synth.seqlen_sweep(n, False)
@@ -194,6 +196,19 @@ def launcher(w, dev_inputs):
     lib = fa.load()
     slopes = synth.alibi_slopes(w.H).cuda() if w.alibi else None
     sp = None if slopes is None else slopes.data_ptr()
+    if w.dtype == synth.E4M3:
+        q, k, v = dev_inputs
+        out = torch.empty(q.shape, device="cuda", dtype=torch.bfloat16)
+        lse = torch.empty((w.B, w.H, w.N), device="cuda", dtype=torch.float32)
+        dq, dk, dv = synth.fp8_factors(w)
+        args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), w.B,
+                w.H, w.N, w.d, 0.0, dq, dk, dv, int(w.causal))
+
+        def go():
+            rc = lib.fa_fwd_fp8(*args, torch.cuda.current_stream().cuda_stream)
+            if rc:
+                raise fa.FaError(rc, "fa_fwd_fp8")
+        return go, (out, lse)
     if w.layout == "varlen":
         q, k, v, cu = dev_inputs
         out = torch.empty_like(q)
@@ -270,6 +285,9 @@ def time_e2e(w, steps, warmup, world):
     dev = [torch.empty_like(t, device="cuda") for t in host]
     if w.layout == "packed":
         o_host = torch.empty((w.B, w.N, w.H, w.d), dtype=host[0].dtype).pin_memory()
+    elif w.dtype == synth.E4M3:
+        o_host = torch.empty(host[0].shape, dtype=torch.bfloat16).pin_memory()
+        factors = synth.fp8_factors(w)
     else:
         o_host = torch.empty_like(host[0]).pin_memory()
     lse_host = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
@@ -283,6 +301,8 @@ def time_e2e(w, steps, warmup, world):
             d.copy_(h, non_blocking=True)
         if w.layout == "packed":
             o, lse = fa.fwd_qkvpacked(dev[0], causal=w.causal)
+        elif w.dtype == synth.E4M3:
+            o, lse = fa.fwd_fp8(dev[0], dev[1], dev[2], *factors, causal=w.causal)
         elif w.layout == "varlen":
             o, lse = fa.fwd_varlen(dev[0], dev[1], dev[2], dev[3], w.N, causal=w.causal,
                                    window_size=w.window, alibi_slopes=slopes)
@@ -337,6 +357,10 @@ class OracleSampler:
         elif w.layout == "varlen":
             q, k, v, cu = synth.make_inputs(w)
             self.cu = cu.numpy()
+        elif w.dtype == synth.E4M3:
+            (q, k, v), f = synth.fp8_inputs(w.B, w.H, w.N, w.d, w.seed, w.sigma_qk, w.sigma_v)
+            q, k, v = (torch.from_numpy(fi * oracle.decode_e4m3(t.view(torch.uint8).numpy()))
+                       for t, fi in zip((q, k, v), f))
         else:
             q, k, v = synth.make_inputs(w)
         self.qkv = tuple(t.double().numpy() for t in (q, k, v))
@@ -414,6 +438,13 @@ def bench_gpu(args, w, key, world, rank, local):
     peaks, peak_src = load_peaks()
     achieved = flops / (ms * 1e-3) / 1e12
     value = world * flops / (ms * 1e-3) / 1e12
+    # e4m3 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (2)
+    ratio = 2.0 if w.dtype == synth.E4M3 else 1.0
+    peak = peaks["bf16_tflops"] * ratio
+    peak_note = (f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json)" if peak_src == "measured"
+                 else "fallback 1.59 PFLOP/s")
+    if ratio != 1.0:
+        peak_note += " x 2 (nominal fp8 / bf16 dense ratio, 4.5 / 2.25 PFLOP/s)"
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
@@ -421,15 +452,14 @@ def bench_gpu(args, w, key, world, rank, local):
         "dtype": synth.DTYPE_NAME[w.dtype], "data": DATA,
         "config": run_config(w, key, world),
         "pct_of_peak": {
-            "measured_burst": round(100 * achieved / peaks["bf16_tflops"], 2),
-            "measured_sustained": round(100 * achieved / peaks["bf16_tflops_sustained"], 2),
-            "nvidia_dense_bf16_datasheet_2250": round(100 * achieved / 2250.0, 2),
+            "measured_burst": round(100 * achieved / peak, 2),
+            "measured_sustained": round(100 * achieved / (peaks["bf16_tflops_sustained"] * ratio), 2),
+            "nvidia_dense_datasheet": round(100 * achieved / (2250.0 * ratio), 2),
             "peaks_source": peak_src},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2),
-                     "peak": peaks["bf16_tflops"], "unit": UNIT,
-                     "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "peak_note": f"{peak_src} dense bf16 burst (MEASURED_PEAKS.json)"
-                                  if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+                     "peak": round(peak, 2), "unit": UNIT,
+                     "frac": round(achieved / peak, 4),
+                     "peak_note": peak_note,
                      "traffic": profiled_traffic(key),
                      "algorithmic_bytes": algorithmic_bytes(w),
                      "kernel": "fa_fwd_kernel", "launches_per_step": 1},
@@ -569,7 +599,7 @@ def run_config(w, key, world):
     return dict(w.describe(), workload_key=key,
                 parallelism=f"replicas{world}" if world > 1 else "single-gpu",
                 global_batch=w.B * world, seq_len=w.N,
-                l2=l2_note(4 * tokens(w) * w.H * w.d * 2))
+                l2=l2_note(algorithmic_bytes(w)))
 
 
 def l2_note(step_bytes):
@@ -581,8 +611,9 @@ def l2_note(step_bytes):
 
 
 def algorithmic_bytes(w):
-    e = 2
-    return 4 * tokens(w) * w.H * w.d * e + 4 * tokens(w) * w.H
+    e = 1 if w.dtype == synth.E4M3 else 2
+    # q, k, v read and o written once (o is bf16 for e4m3 inputs), fp32 LSE
+    return (3 * e + 2) * tokens(w) * w.H * w.d + 4 * tokens(w) * w.H
 
 
 def main():

@@ -41,7 +41,7 @@ struct DeviceState {
   bool ready = false;
   bool is_sm100 = false;
   int sm_count = 0;
-  bool attr_set[12] = {};
+  bool attr_set[18] = {};
   bool bwd_attr_set[8] = {false, false, false, false, false, false, false, false};
   float* bwd_scratch = nullptr;  // this device's g_bwd_scratch
 };
@@ -87,35 +87,44 @@ int device_state(DeviceState** out, int* dev_out) {
 }
 
 // 4-D view (d, N, H, B) of one operand with element strides (1, sn, sh, sb);
-// box of 64 elements (128 bytes) x `rows` rows, 128-byte swizzle, zero fill.
+// box of 128 bytes (64 16-bit or 128 8-bit elements) x `rows` rows, 128-byte
+// swizzle, zero fill.  e4m3 operands are mapped as bytes.
 int encode_operand(CUtensorMap* map, const void* ptr, int dtype, int d, int N, int H, int B,
                    long long sn, long long sh, long long sb, int rows) {
+  const int eb = dtype == FA_E4M3 ? 1 : 2;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)H, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)sn * 2, (cuuint64_t)sh * 2, (cuuint64_t)sb * 2};
-  const cuuint32_t box[4] = {64, (cuuint32_t)rows, 1, 1};
+  const cuuint64_t strides[3] = {(cuuint64_t)sn * eb, (cuuint64_t)sh * eb, (cuuint64_t)sb * eb};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), (cuuint32_t)rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUtensorMapDataType t =
-      dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType t = dtype == FA_E4M3   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                : dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUresult r = g_encode(map, t, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// Kernel configuration per head dim: (Q tiles per work tile, K/V ring stages).
-template <int HD> struct Pick;
-template <> struct Pick<64> { static constexpr int QS = 2, KVS = 10; };
-template <> struct Pick<128> { static constexpr int QS = 2, KVS = 4; };
-template <> struct Pick<256> { static constexpr int QS = 1, KVS = 2; };
+// Kernel configuration per head dim and element size: (Q tiles per work
+// tile, K/V ring stages).  e4m3 tiles are half the bytes, so the ring is
+// deeper; their MMAs take half the time.
+template <int HD, int ELT> struct Pick;
+template <int ELT> struct Pick<64, ELT> { static constexpr int QS = 2, KVS = 10; };
+template <> struct Pick<128, kF16> { static constexpr int QS = 2, KVS = 4; };
+template <> struct Pick<128, kBF16> { static constexpr int QS = 2, KVS = 4; };
+template <> struct Pick<128, kE4M3> { static constexpr int QS = 2, KVS = 10; };
+template <> struct Pick<256, kF16> { static constexpr int QS = 1, KVS = 2; };
+template <> struct Pick<256, kBF16> { static constexpr int QS = 1, KVS = 2; };
+template <> struct Pick<256, kE4M3> { static constexpr int QS = 1, KVS = 5; };
 
 int q_tiles_for(int d) { return d == 256 ? 1 : 2; }
 
-template <int HD, bool BF16, bool ALIBI>
+template <int HD, int ELT, bool ALIBI>
 int launch(FwdParams& p, DeviceState& st, cudaStream_t stream) {
-  constexpr int QS = Pick<HD>::QS, KVS = Pick<HD>::KVS;
-  using C = FwdCfg<HD, QS, KVS, BF16>;
-  auto kernel = fa_fwd_kernel<HD, QS, KVS, BF16, ALIBI>;
-  const int slot = (HD == 64 ? 0 : HD == 128 ? 2 : 4) + (BF16 ? 1 : 0) + (ALIBI ? 6 : 0);
+  constexpr int QS = Pick<HD, ELT>::QS, KVS = Pick<HD, ELT>::KVS;
+  using C = FwdCfg<HD, QS, KVS, ELT>;
+  auto kernel = fa_fwd_kernel<HD, QS, KVS, ELT, ALIBI>;
+  const int slot = ((HD == 64 ? 0 : HD == 128 ? 1 : 2) * 3 + ELT) * 2 + (ALIBI ? 1 : 0);
   if (!st.attr_set[slot]) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_BYTES) != cudaSuccess) {
@@ -143,8 +152,9 @@ int normalize_window(int N, int causal, int* left, int* right) {
 }
 
 int check_common(int B, int H, int N, int d, float* scale, int causal, int dtype) {
-  if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+  if (dtype != FA_FP16 && dtype != FA_BF16 && dtype != FA_E4M3) return FA_ERR_DTYPE;
   if (d != 64 && d != 128 && d != 256) return FA_ERR_HEADDIM;
+  if (dtype == FA_E4M3 && d == 64) return FA_ERR_HEADDIM;
   if (B < 1 || H < 1 || N < 1) return FA_ERR_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_ARG;
   if (!std::isfinite(*scale) || *scale < 0.f) return FA_ERR_ARG;
@@ -173,11 +183,23 @@ struct Problem {
   int window_left, window_right;
   const float* alibi;
   const int* cu_seqlens;
+  float qk_descale, v_descale;  // e4m3: dequantisation factors; 1 otherwise
 };
 
-template <int HD, bool BF16>
+template <int HD, int ELT>
 int launch_masks(FwdParams& p, bool alibi, DeviceState& st, cudaStream_t stream) {
-  return alibi ? launch<HD, BF16, true>(p, st, stream) : launch<HD, BF16, false>(p, st, stream);
+  return alibi ? launch<HD, ELT, true>(p, st, stream) : launch<HD, ELT, false>(p, st, stream);
+}
+
+template <int HD>
+int launch_elt(FwdParams& p, int dtype, bool alibi, DeviceState& st, cudaStream_t stream) {
+  if (dtype == FA_BF16) return launch_masks<HD, kBF16>(p, alibi, st, stream);
+  if (dtype == FA_FP16) return launch_masks<HD, kF16>(p, alibi, st, stream);
+  if constexpr (HD >= 128) {
+    // e4m3: no ALiBi variant (fa_fwd_fp8 takes none)
+    if (!alibi) return launch<HD, kE4M3, false>(p, st, stream);
+  }
+  return FA_ERR_ARG;
 }
 
 int run(const Problem& pr, cudaStream_t stream) {
@@ -216,23 +238,18 @@ int run(const Problem& pr, cudaStream_t stream) {
   p.window_left = pr.window_left;
   p.window_right = pr.window_right;
   p.alibi_slopes = pr.alibi;
-  p.scale_log2 = pr.scale * 1.4426950408889634f;
+  p.scale_log2 = pr.scale * pr.qk_descale * 1.4426950408889634f;
+  p.o_scale = pr.v_descale;
   const int rows_per_tile = 128 * q_tiles_for(pr.d);
   p.num_qblocks = (pr.N + rows_per_tile - 1) / rows_per_tile;
   p.num_tiles = pr.B * pr.H * p.num_qblocks;
   p.wait_limit_ns = kWaitLimitNs;
 
-  const bool bf16 = pr.dtype == FA_BF16, alibi = pr.alibi != nullptr;
+  const bool alibi = pr.alibi != nullptr;
   switch (pr.d) {
-    case 64:
-      return bf16 ? launch_masks<64, true>(p, alibi, *st, stream)
-                  : launch_masks<64, false>(p, alibi, *st, stream);
-    case 128:
-      return bf16 ? launch_masks<128, true>(p, alibi, *st, stream)
-                  : launch_masks<128, false>(p, alibi, *st, stream);
-    default:
-      return bf16 ? launch_masks<256, true>(p, alibi, *st, stream)
-                  : launch_masks<256, false>(p, alibi, *st, stream);
+    case 64: return launch_elt<64>(p, pr.dtype, alibi, *st, stream);
+    case 128: return launch_elt<128>(p, pr.dtype, alibi, *st, stream);
+    default: return launch_elt<256>(p, pr.dtype, alibi, *st, stream);
   }
 }
 
@@ -251,6 +268,7 @@ Problem bhnd_problem(const void* q, const void* k, const void* v, void* o, float
   pr.map_rows = N;
   pr.map_batches = B;
   pr.window_left = pr.window_right = -1;
+  pr.qk_descale = pr.v_descale = 1.f;
   return pr;
 }
 
@@ -307,6 +325,7 @@ int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse,
                int N, int d, float scale, int causal, int window_left, int window_right,
                const float* alibi_slopes, int dtype, struct CUstream_st* stream) {
   if (!q || !k || !v || !o) return FA_ERR_ARG;
+  if (dtype == FA_E4M3) return FA_ERR_DTYPE;  // e4m3 goes through fa_fwd_fp8
   int rc = check_common(B, H, N, d, &scale, causal, dtype);
   if (rc != FA_OK) return rc;
   if ((rc = normalize_window(N, causal, &window_left, &window_right)) != FA_OK) return rc;
@@ -331,6 +350,7 @@ int fa_fwd_qkvpacked_ext(const void* qkv, void* o, float* lse, int B, int N, int
                          struct CUstream_st* stream) {
   if (!qkv || !o) return FA_ERR_ARG;
   if (!(dropout_p == 0.0f)) return std::isnan(dropout_p) ? FA_ERR_ARG : FA_ERR_UNSUPPORTED;
+  if (dtype == FA_E4M3) return FA_ERR_DTYPE;
   int rc = check_common(B, H, N, d, &scale, causal, dtype);
   if (rc != FA_OK) return rc;
   if ((rc = normalize_window(N, causal, &window_left, &window_right)) != FA_OK) return rc;
@@ -349,11 +369,31 @@ int fa_fwd_qkvpacked(const void* qkv, void* o, float* lse, int B, int N, int H, 
                               dtype, stream);
 }
 
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+               int N, int d, float scale, float descale_q, float descale_k, float descale_v,
+               int causal, struct CUstream_st* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_ARG;
+  int rc = check_common(B, H, N, d, &scale, causal, FA_E4M3);
+  if (rc != FA_OK) return rc;
+  for (float f : {descale_q, descale_k, descale_v})
+    if (!std::isfinite(f) || !(f > 0.f)) return FA_ERR_ARG;
+  if (!std::isfinite(scale * descale_q * descale_k) || !(scale * descale_q * descale_k > 0.f))
+    return FA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned4(lse))
+    return FA_ERR_ALIGN;
+  Problem pr = bhnd_problem(q, k, v, o, lse, B, H, N, d, scale, causal, FA_E4M3);
+  pr.qk_descale = descale_q * descale_k;
+  pr.v_descale = descale_v;
+  if (causal) pr.window_right = 0;
+  return run(pr, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int* cu_seqlens, int batch, int max_seqlen, int total, int H, int d,
                   float scale, int causal, int window_left, int window_right,
                   const float* alibi_slopes, int dtype, struct CUstream_st* stream) {
   if (!q || !k || !v || !o || !cu_seqlens) return FA_ERR_ARG;
+  if (dtype == FA_E4M3) return FA_ERR_DTYPE;
   int rc = check_common(batch, H, max_seqlen, d, &scale, causal, dtype);
   if (rc != FA_OK) return rc;
   if (total < 1 || (long long)total * H * d > (1ll << 46)) return FA_ERR_ARG;

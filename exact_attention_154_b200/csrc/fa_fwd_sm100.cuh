@@ -69,6 +69,11 @@ __host__ __device__ constexpr int poly_pairs_per8() {
 #endif
 }
 
+// Operand element types of the forward: fp16 and bf16 (kind::f16 MMAs, P and
+// O in the same type) and fp8 e4m3 (kind::f8f6f4 MMAs, P in e4m3, O in bf16).
+enum Elt : int { kF16 = 0, kBF16 = 1, kE4M3 = 2 };
+__host__ __device__ constexpr int elt_bytes(int elt) { return elt == kE4M3 ? 1 : 2; }
+
 // Error word written by a kernel whose bounded wait ran out: 0 = none,
 // otherwise (role << 8) | site, first writer wins.
 __device__ unsigned int g_fa_watchdog = 0u;
@@ -104,7 +109,8 @@ struct FwdParams {
   // mask arrives here as window_right = 0.
   int window_left, window_right;
   const float* alibi_slopes;  // [H]: the scaled score gets -slope[h] * |i - j|; or nullptr
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (e4m3: times the q and k descale factors)
+  float o_scale;     // factor on O / l: 1, or the v descale factor (e4m3)
   int num_qblocks;   // query blocks per (b, h) (of the longest sequence)
   int num_tiles;     // B * H * num_qblocks
   unsigned long long wait_limit_ns;
@@ -129,15 +135,23 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
   }
 }
 
-template <int HD, int QS, int KVS, bool BF16>
+template <int HD, int QS, int KVS, int ELT>
 struct FwdCfg {
   static_assert(HD == 64 || HD == 128 || HD == 256, "head dim");
   static_assert(QS == 1 || QS == 2, "Q tiles per work tile");
-  static constexpr int CHUNKS = HD / 64;          // 128-byte column chunks per row
-  static constexpr int CHUNK_BYTES = 128 * 128;   // one chunk of a 128-row tile
+  static_assert(ELT != kE4M3 || HD >= 128, "fp8 rows must fill a 128-byte swizzle row");
+  static constexpr int EB = elt_bytes(ELT);         // bytes per element
+  static constexpr int BOX = 128 / EB;              // elements per 128-byte row chunk
+  static constexpr int CHUNKS = HD * EB / 128;      // 128-byte column chunks per row
+  static constexpr int CHUNK_BYTES = 128 * 128;     // one chunk of a 128-row tile
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;
-  // one 128 x 128 16-bit P tile, used by the Q tiles in turn
-  static constexpr int P_TILE_BYTES = (BN / 64) * CHUNK_BYTES;
+  // Every MMA K-step takes 32 bytes of each operand row: 16 fp16 / bf16 or
+  // 32 e4m3 elements.
+  static constexpr int KSTEP = 32 / EB;
+  static constexpr int S_KSTEPS = HD / KSTEP;       // S = Q K^T
+  static constexpr int PV_KSTEPS = BN / KSTEP;      // O += P V, over the 128 keys
+  // one 128 x 128 P tile (16-bit, or e4m3), used by the Q tiles in turn
+  static constexpr int P_TILE_BYTES = (BN * EB / 128) * CHUNK_BYTES;
   // two softmax warpgroups per Q tile: key columns 0-63 and 64-127 of the
   // same 128 rows
   static constexpr int SOFTMAX_WGS = 2 * QS;
@@ -287,6 +301,13 @@ __device__ __forceinline__ int tile_of(int round, int cta, int G) {
   return round * G + ((round & 1) ? (G - 1 - cta) : cta);
 }
 
+// Two e4m3 codes (round to nearest, saturating) in 16 bits: lo in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   if constexpr (BF16) {
@@ -305,9 +326,9 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // ------------------------------------------------------------------ roles
-template <int HD, int QS, int KVS, bool BF16>
+template <int HD, int QS, int KVS, int ELT>
 __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* abort_flag) {
-  using C = FwdCfg<HD, QS, KVS, BF16>;
+  using C = FwdCfg<HD, QS, KVS, ELT>;
   const uint32_t bars = base + C::BAR_OFF;
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0, q_count = 0;
@@ -323,7 +344,7 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
 #pragma unroll
     for (int c = 0; c < C::CHUNKS; ++c)
       tma_load_4d(base + C::SKV_OFF + slot * C::TILE_BYTES + c * C::CHUNK_BYTES, map, full,
-                  c * 64, ti.row0 + row0, ti.h, ti.bc);
+                  c * C::BOX, ti.row0 + row0, ti.h, ti.bc);
     ++kv_count;
     return true;
   };
@@ -346,7 +367,7 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
 #pragma unroll
       for (int c = 0; c < C::CHUNKS; ++c)
         tma_load_4d(base + C::SQ_OFF + s * C::TILE_BYTES + c * C::CHUNK_BYTES, &p.tmap_q,
-                    bars + 8 * C::B_Q_FULL, c * 64, ti.row0 + ti.q0 + s * BM, ti.h, ti.bc);
+                    bars + 8 * C::B_Q_FULL, c * C::BOX, ti.row0 + ti.q0 + s * BM, ti.h, ti.bc);
     ++q_count;
     for (int jj = 0; ok && jj < ti.n_u; ++jj) {
       const int j = ti.lo_u + jj;
@@ -378,12 +399,13 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
 
 // S thread, per work tile: S_s(0) for every Q tile s, then S_s(j+1) once the
 // softmax of tile s has read S_s(j) out of TMEM.
-template <int HD, int QS, int KVS, bool BF16>
+template <int HD, int QS, int KVS, int ELT>
 __device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
                            volatile int* abort_flag) {
-  using C = FwdCfg<HD, QS, KVS, BF16>;
+  using C = FwdCfg<HD, QS, KVS, ELT>;
   const uint32_t bars = base + C::BAR_OFF;
-  const uint32_t idesc_qk = f16_idesc(BF16, BM, BN, false);
+  const uint32_t idesc_qk =
+      ELT == kE4M3 ? e4m3_idesc(BM, BN, false) : f16_idesc(ELT == kBF16, BM, BN, false);
   const unsigned long long lim = p.wait_limit_ns;
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0, q_count = 0;
@@ -412,9 +434,12 @@ __device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const uint32_t kb = sw128_desc_lo(base + C::SKV_OFF + kslot * C::TILE_BYTES, 16);
     const uint32_t d_tmem = tmem + C::s_col(s);
 #pragma unroll
-    for (int kk = 0; kk < HD / 16; ++kk) {
+    for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
       const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
-      mma_ss(d_tmem, desc_from_lo(qa + off), desc_from_lo(kb + off), idesc_qk, kk > 0 ? 1u : 0u);
+      if constexpr (ELT == kE4M3)
+        mma_ss_f8(d_tmem, desc_from_lo(qa + off), desc_from_lo(kb + off), idesc_qk, kk > 0 ? 1u : 0u);
+      else
+        mma_ss(d_tmem, desc_from_lo(qa + off), desc_from_lo(kb + off), idesc_qk, kk > 0 ? 1u : 0u);
     }
     tc_commit(bars + 8 * (C::B_S_FULL + s));
     ++s_issued[s];
@@ -457,12 +482,13 @@ __device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
 // then tile 1, each once the softmax has written P_s(j) into the shared P
 // buffer; after each product the buffer is handed to the tile that uses it
 // next (which also tells that tile's softmax that O_s holds the product).
-template <int HD, int QS, int KVS, bool BF16>
+template <int HD, int QS, int KVS, int ELT>
 __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
                             volatile int* abort_flag) {
-  using C = FwdCfg<HD, QS, KVS, BF16>;
+  using C = FwdCfg<HD, QS, KVS, ELT>;
   const uint32_t bars = base + C::BAR_OFF;
-  const uint32_t idesc_pv = f16_idesc(BF16, BM, HD, true);
+  const uint32_t idesc_pv =
+      ELT == kE4M3 ? e4m3_idesc(BM, HD, true) : f16_idesc(ELT == kBF16, BM, HD, true);
   const unsigned long long lim = p.wait_limit_ns;
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0;
@@ -477,18 +503,25 @@ __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   auto issue_pv = [&](int s, int vslot, bool accumulate, int nxt) -> bool {
     const uint32_t vb = sw128_desc_lo(base + C::SKV_OFF + vslot * C::TILE_BYTES, C::CHUNK_BYTES);
     const uint32_t d_tmem = tmem + (s ? C::O_COL1 : C::O_COL0);
+    // Byte offset of the first key of half h in a P row: 64 keys of 16 bits
+    // fill one 128-byte chunk, 64 e4m3 keys half of one.
+    constexpr int HALF_STEPS = C::PV_KSTEPS / 2;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       if (!wait_phase(bars + 8 * (C::B_P_FULL + half), p_par, abort_flag, lim,
                       (kRoleMma << 8) | kSitePFull))
         return false;
       tc_fence_after_sync();
+      const int half_off = C::EB == 2 ? half * C::CHUNK_BYTES : half * 64;
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int kk = half * 4 + k4;
-        mma_ss(d_tmem, desc_from_lo(pa + ((half * C::CHUNK_BYTES + k4 * 32) >> 4)),
-               desc_from_lo(vb + ((kk * 16 * 128) >> 4)), idesc_pv,
-               (accumulate || kk > 0) ? 1u : 0u);
+      for (int k = 0; k < HALF_STEPS; ++k) {
+        const int kk = half * HALF_STEPS + k;
+        const uint64_t a = desc_from_lo(pa + ((half_off + k * 32) >> 4));
+        const uint64_t b = desc_from_lo(vb + ((kk * C::KSTEP * 128) >> 4));
+        if constexpr (ELT == kE4M3)
+          mma_ss_f8(d_tmem, a, b, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        else
+          mma_ss(d_tmem, a, b, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
       }
       tc_commit(bars + 8 * (C::B_P_FREE + 2 * nxt + half));
     }
@@ -589,7 +622,9 @@ __device__ __forceinline__ void store_p_chunk(uint32_t chunk_base, int r, const 
 // POLY8 of every 8 argument pairs go through exp2_poly2, the rest through ex2.
 // The row sum goes into four independent packed accumulators, so the adds
 // form four short dependency chains instead of one long one.
-template <bool BF16, int POLY8>
+// 16-bit P: pk[q] holds keys 2q, 2q+1.  e4m3 P: pk[q / 2] holds keys
+// 4(q/2) .. 4(q/2)+3, low byte first (so pk covers 16 words, not 32).
+template <int ELT, int POLY8>
 __device__ __forceinline__ void softmax_chunk(const float* sv, float sl2, float neg_ref,
                                               uint32_t* pk, float2 (&acc)[4]) {
 #pragma unroll
@@ -604,17 +639,38 @@ __device__ __forceinline__ void softmax_chunk(const float* sv, float sl2, float 
       e.y = ex2(x.y);
     }
     acc[q & 3] = __fadd2_rn(acc[q & 3], e);
-    pk[q] = pack2<BF16>(e.x, e.y);
+    if constexpr (ELT == kE4M3) {
+      const uint32_t h = pack_e4m3x2(e.x, e.y);
+      if (q & 1)
+        pk[q / 2] |= h << 16;
+      else
+        pk[q / 2] = h;
+    } else {
+      pk[q] = pack2<ELT == kBF16>(e.x, e.y);
+    }
   }
+}
+
+// Writes 64 e4m3 keys of one P row (16 words) into its half (bytes 64 hf ..
+// 64 hf + 63) of the row's 128-byte swizzled line: 16-byte group u of the
+// line at position u ^ (r % 8).
+__device__ __forceinline__ void store_p_half_e4m3(uint32_t p_base, int r, int hf,
+                                                  const uint32_t* pk) {
+  const uint32_t row = p_base + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    st_shared_v4(row + ((static_cast<uint32_t>(4 * hf + u) ^ (r & 7u)) << 4), pk[4 * u],
+                 pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
 }
 
 // ALIBI: the scaled score of key j gets -slope[h] * |i - j| (in the log2
 // domain, -slope[h] * log2(e) * |i - j|) before the row max is taken.
-template <int HD, int QS, int KVS, bool BF16, bool ALIBI>
+template <int HD, int QS, int KVS, int ELT, bool ALIBI>
 __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
                              volatile int* abort_flag) {
-  using C = FwdCfg<HD, QS, KVS, BF16>;
-  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  using C = FwdCfg<HD, QS, KVS, ELT>;
+  constexpr bool OUT_BF16 = ELT != kF16;  // e4m3 inputs give a bf16 output
+  using T = typename std::conditional<OUT_BF16, __nv_bfloat16, __half>::type;
   constexpr int HD2 = HD / 2;                 // O columns each group of a tile owns
   const uint32_t bars = base + C::BAR_OFF;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -625,7 +681,8 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const uint32_t lane_base = tmem + ((static_cast<uint32_t>(warp % 4) * 32u) << 16);
   const uint32_t s_col = C::s_col(s) + 64u * hf;
   const uint32_t o_col = (s ? C::O_COL1 : C::O_COL0) + HD2 * hf;
-  const uint32_t sp = base + C::SP_OFF + hf * C::CHUNK_BYTES;  // this group's half of P
+  // this group's half of P: its own chunk (16-bit), or half of each line (e4m3)
+  const uint32_t sp = base + C::SP_OFF + (C::EB == 2 ? hf * C::CHUNK_BYTES : 0);
   float* xch = reinterpret_cast<float*>(
       __cvta_shared_to_generic(base + C::XCH_OFF));
   float* x_mine = xch + (s * 2 + hf) * 128;
@@ -725,13 +782,15 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
 
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
-      uint32_t pk[32];
+      constexpr int PK_WORDS = 32 * C::EB / 2;  // words of P per 32 keys, times 2
+      uint32_t pk[PK_WORDS];
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         if (need_mask)
-          softmax_chunk<BF16, 0>(sv + 32 * c, sl2e, neg_ref, pk + 16 * c, acc);
+          softmax_chunk<ELT, 0>(sv + 32 * c, sl2e, neg_ref, pk + (PK_WORDS / 2) * c, acc);
         else
-          softmax_chunk<BF16, poly_pairs_per8<HD>()>(sv + 32 * c, sl2e, neg_ref, pk + 16 * c, acc);
+          softmax_chunk<ELT, poly_pairs_per8<HD>()>(sv + 32 * c, sl2e, neg_ref,
+                                                    pk + (PK_WORDS / 2) * c, acc);
       }
       // This group's half of the P buffer is this tile's turn: the previous
       // user's K-steps that read it have run.
@@ -769,7 +828,10 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         __syncwarp();
         if (lane == 0) mbar_arrive(bars + 8 * C::B_P_FULL);
       }
-      store_p_chunk(sp, r, pk);
+      if constexpr (ELT == kE4M3)
+        store_p_half_e4m3(sp, r, hf, pk);
+      else
+        store_p_chunk(sp, r, pk);
       // make the generic-proxy stores visible to the tensor core
       fence_proxy_async_smem();
       tc_fence_before_sync();
@@ -791,7 +853,7 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     if (!group_meet()) return;
     const float l_row = l + x_other[r];
     if (!group_meet()) return;  // both have read before the slots are reused
-    const float inv_l = 1.f / l_row;
+    const float inv_l = p.o_scale / l_row;
     const long long trow = static_cast<long long>(ti.row0) + row;  // tensor row
     const bool store = row < ti.len && trow < p.rows_total;
     T* orow = reinterpret_cast<T*>(p.o) + ti.bc * p.o_stride_b + ti.h * p.o_stride_h +
@@ -804,7 +866,8 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
       for (int i = 0; i < 16; ++i)
-        wp[i] = pack2<BF16>(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+        wp[i] = pack2<OUT_BF16>(__uint_as_float(ov[2 * i]) * inv_l,
+                                __uint_as_float(ov[2 * i + 1]) * inv_l);
       if (store) {
         uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
@@ -820,10 +883,10 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   }
 }
 
-template <int HD, int QS, int KVS, bool BF16, bool ALIBI>
-__global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
+template <int HD, int QS, int KVS, int ELT, bool ALIBI>
+__global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, ELT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<HD, QS, KVS, BF16>;
+  using C = FwdCfg<HD, QS, KVS, ELT>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -884,13 +947,13 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, BF16>::THREADS, 1)
   }
 
   if (warp < C::SOFTMAX_WARPS) {
-    softmax_role<HD, QS, KVS, BF16, ALIBI>(p, base, tmem, abort_flag);
+    softmax_role<HD, QS, KVS, ELT, ALIBI>(p, base, tmem, abort_flag);
   } else if (warp == C::PRODUCER_WARP) {
-    if (lane == 0) producer_role<HD, QS, KVS, BF16>(p, base, abort_flag);
+    if (lane == 0) producer_role<HD, QS, KVS, ELT>(p, base, abort_flag);
   } else if (warp == C::MMA_S_WARP) {
-    if (lane == 0) mma_s_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
+    if (lane == 0) mma_s_role<HD, QS, KVS, ELT>(p, base, tmem, abort_flag);
   } else if (warp == C::MMA_PV_WARP) {
-    if (lane == 0) mma_pv_role<HD, QS, KVS, BF16>(p, base, tmem, abort_flag);
+    if (lane == 0) mma_pv_role<HD, QS, KVS, ELT>(p, base, tmem, abort_flag);
   }  // the last warp has no role
 
   tc_fence_before_sync();

@@ -33,6 +33,7 @@ SIGNATURES = {
     "fa_fwd_ext": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I, _I, _FP, _I, _VP]),
     "fa_fwd_qkvpacked_ext": (_I, [_VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _F, _I, _I, _FP, _I,
                                   _VP]),
+    "fa_fwd_fp8": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _F, _F, _F, _I, _VP]),
     "fa_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _I, _FP,
                            _I, _VP]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _F, _I, _I,
@@ -216,6 +217,34 @@ def fwd_qkvpacked(qkv: torch.Tensor, dropout_p: float = 0.0, softmax_scale: floa
             float(dropout_p), left, right, slopes_ptr, _DT[qkv.dtype], _stream_ptr(qkv))
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd_qkvpacked_ext")
+    return out, lse
+
+
+def fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, descale_q: float,
+            descale_k: float, descale_v: float, scale: float | None = None,
+            causal: bool = False, return_lse: bool = True):
+    """Forward on fp8 e4m3 ``[B, H, N, d]`` tensors (torch.float8_e4m3fn, or
+    uint8 holding the codes) with per-tensor dequantisation factors: the real
+    operands are ``descale_x * x``.  Returns ``(O bf16 [B, H, N, d], LSE)``."""
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dtype not in (torch.float8_e4m3fn, torch.uint8) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous float8_e4m3fn (or uint8) tensor")
+    if not (q8.shape == k8.shape == v8.shape) or q8.dim() != 4:
+        raise ValueError("q8, k8, v8 must share one [B, H, N, d] shape")
+    B, H, N, d = q8.shape
+    dev = same_device([("q8", q8), ("k8", k8), ("v8", v8)])
+    out = torch.empty((B, H, N, d), device=dev, dtype=torch.bfloat16)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32) if return_lse else None
+    with _on(dev):
+        rc = load().fa_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), out.data_ptr(),
+                               None if lse is None else lse.data_ptr(), B, H, N, d,
+                               0.0 if scale is None else float(scale), float(descale_q),
+                               float(descale_k), float(descale_v), int(bool(causal)),
+                               _stream_ptr(q8))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_fp8")
     return out, lse
 
 

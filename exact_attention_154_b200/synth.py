@@ -26,9 +26,9 @@ from dataclasses import dataclass, field
 import numpy as np
 import torch
 
-FP16, BF16 = 0, 1
-TORCH_DTYPE = {FP16: torch.float16, BF16: torch.bfloat16}
-DTYPE_NAME = {FP16: "f16", BF16: "bf16"}
+FP16, BF16, E4M3 = 0, 1, 2
+TORCH_DTYPE = {FP16: torch.float16, BF16: torch.bfloat16, E4M3: torch.float8_e4m3fn}
+DTYPE_NAME = {FP16: "f16", BF16: "bf16", E4M3: "e4m3"}
 
 
 @dataclass(frozen=True)
@@ -169,6 +169,13 @@ def varlen_mix_causal() -> Workload:
                     BF16, True, 62, layout="varlen", lengths=lengths)
 
 
+def fp8_sweep_n4096(causal: bool = False) -> Workload:
+    """The N = 4096 sweep shape on fp8 e4m3 operands (per-tensor factors)."""
+    tag = "causal" if causal else "non-causal"
+    return Workload(f"fp8 e4m3 fwd B=4,H=16,N=4096,d=128 {tag}, bf16 output", 4, 16, 4096, 128,
+                    E4M3, causal, 63 + int(causal))
+
+
 def all_workloads() -> list[Workload]:
     w = [single_head_n256(), packed_qkv_b2_n256_h12(), many_heads_causal_n2048()]
     for n in SWEEP_N:
@@ -183,8 +190,11 @@ def make_inputs(w: Workload):
 
     ``bhnd`` -> ``(q, k, v)`` each [B, H, N, d]; ``packed`` -> ``(qkv,)`` of
     shape [B, N, 3, H, d] (index 0/1/2 of axis 2 = q/k/v); ``varlen`` ->
-    ``(q, k, v, cu_seqlens)`` with q, k, v [total, H, d].
+    ``(q, k, v, cu_seqlens)`` with q, k, v [total, H, d]; e4m3 workloads
+    ``(q8, k8, v8)`` (their factors: :func:`fp8_factors`).
     """
+    if w.dtype == E4M3:
+        return fp8_inputs(w.B, w.H, w.N, w.d, w.seed, w.sigma_qk, w.sigma_v)[0]
     g = torch.Generator().manual_seed(w.seed)
     dt = TORCH_DTYPE[w.dtype]
     if w.layout == "varlen":
@@ -239,6 +249,32 @@ def packed_lengths(lengths, H, d, dtype, seed, sigma_qk=1.0, sigma_v=1.0, extra_
     v = torch.randn((total, H, d), generator=g, dtype=torch.float32) * sigma_v
     cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
     return q.to(dt), k.to(dt), v.to(dt), cu
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor fp8 quantisation of an fp32 tensor: descale = amax / 448
+    rounded to fp32, codes = round-to-nearest e4m3 of x / descale (torch's
+    float8_e4m3fn conversion).  Returns (codes as float8_e4m3fn, descale)."""
+    amax = float(x.abs().max())
+    descale = float(torch.tensor(max(amax, 1e-30) / 448.0, dtype=torch.float32))
+    return (x / descale).to(torch.float8_e4m3fn), descale
+
+
+def fp8_factors(w: Workload):
+    """The (descale_q, descale_k, descale_v) of an e4m3 workload's inputs."""
+    return fp8_inputs(w.B, w.H, w.N, w.d, w.seed, w.sigma_qk, w.sigma_v)[1]
+
+
+def fp8_inputs(B, H, N, d, seed, sigma_qk=1.0, sigma_v=1.0):
+    """[B, H, N, d] fp8 q, k, v and their descale factors: the draws of
+    :func:`make_inputs` (fp32 randn times sigma), each quantised per tensor by
+    :func:`quantize_e4m3`.  Returns ``((q8, k8, v8), (dq, dk, dv))``."""
+    g = torch.Generator().manual_seed(seed)
+    shape = (B, H, N, d)
+    xs = [torch.randn(shape, generator=g, dtype=torch.float32) * s
+          for s in (sigma_qk, sigma_qk, sigma_v)]
+    out = [quantize_e4m3(x) for x in xs]
+    return tuple(c for c, _ in out), tuple(f for _, f in out)
 
 
 def random_inputs(B, H, N, d, dtype, seed, sigma_qk=1.0, sigma_v=1.0):

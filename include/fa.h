@@ -49,7 +49,7 @@ enum fa_status {
   FA_ERR_ARG = -1,         /* null pointer, B/H/N < 1, bad scale, size overflow */
   FA_ERR_ALIGN = -2,       /* a tensor pointer is not 16-byte aligned */
   FA_ERR_HEADDIM = -3,     /* d is not 64, 128 or 256 */
-  FA_ERR_DTYPE = -4,       /* dtype is not FA_FP16 or FA_BF16 */
+  FA_ERR_DTYPE = -4,       /* dtype is not FA_FP16 or FA_BF16 (or FA_E4M3 where taken) */
   FA_ERR_UNSUPPORTED = -5, /* dropout_p != 0 */
   FA_ERR_CUDA = -6,        /* a CUDA runtime / driver call failed */
   FA_ERR_TIMEOUT = -7,     /* a kernel gave up on a bounded wait */
@@ -57,7 +57,8 @@ enum fa_status {
   FA_ERR_SEQLENS = -9      /* (fa_device_status) a kernel met cu_seqlens out of range */
 };
 
-enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1 };
+/* FA_E4M3 (fp8 e4m3 operands) is accepted by fa_fwd_fp8 only. */
+enum fa_dtype { FA_FP16 = 0, FA_BF16 = 1, FA_E4M3 = 2 };
 
 /*
  * Attention forward on separate Q, K, V.
@@ -128,6 +129,34 @@ int fa_fwd_qkvpacked_ext(const void *qkv, void *o, float *lse, int B, int N, int
                          float scale, int causal, float dropout_p, int window_left,
                          int window_right, const float *alibi_slopes, int dtype,
                          struct CUstream_st *stream);
+
+/*
+ * Forward on fp8 (e4m3) Q, K, V with per-tensor dequantisation factors: the
+ * low-precision inference path of item 4, "低精度推理支持" (INT8 / FP8), of
+ * "flash-attention与TensorRT 10集成" (blog.gitcode.com).  The page names FP8
+ * inference without fixing a format; the reading taken here:
+ *
+ *   q, k, v   : [B, H, N, d] contiguous e4m3 codes (1 byte each: sign, 4
+ *               exponent bits with bias 7, 3 mantissa bits, no infinities;
+ *               the OCP "E4M3FN" format), read only
+ *   descale_q, descale_k, descale_v : the real tensors are descale_x * x;
+ *               finite and > 0
+ *   o         : [B, H, N, d] contiguous bf16 (written)
+ *   lse       : [B, H, N] fp32 (written), or NULL
+ *   d         : 128 or 256 (a row must fill a 128-byte line; else FA_ERR_HEADDIM)
+ *   scale, causal, stream : as fa_fwd
+ *
+ * It computes O = softmax(scale * (descale_q Q)(descale_k K)^T [+ causal])
+ * (descale_v V) and its logsumexp.  S = Q K^T is formed from the e4m3 codes
+ * on the tensor cores with fp32 accumulation; the softmax weights P are
+ * rounded to e4m3 (3 mantissa bits, values near or below 2^-9 of the row's
+ * reference flush to zero) before P V, the row sum uses the unrounded fp32
+ * weights.  That rounding, not the inputs, sets the output error: see the
+ * per-element bound the tests state.
+ */
+int fa_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse, int B, int H,
+               int N, int d, float scale, float descale_q, float descale_k, float descale_v,
+               int causal, struct CUstream_st *stream);
 
 /*
  * Forward over a batch of sequences of different lengths packed back to back

@@ -23,6 +23,10 @@ Three independent implementations live here:
 * :func:`attention_varlen` -- sequences of different lengths packed back to
   back (``[total, H, d]`` with ``cu_seqlens`` offsets): the definition applied
   to each sequence on its own, pinned in ``tests/test_oracle_varlen_pins.py``.
+* :func:`decode_e4m3` and :func:`attention_fp8` -- fp8 (e4m3) operands with
+  per-tensor dequantisation factors: the codes decoded by the format's
+  definition, then the plain definition on the dequantised values; pinned in
+  ``tests/test_oracle_fp8_pins.py``.
 * :func:`attention_bwd` -- the gradient of the plain definition with respect
   to q, k, v (chain rule written out in ``fa_oracle.c``), pinned in
   ``tests/test_oracle_bwd_pins.py`` by central finite differences of
@@ -30,7 +34,7 @@ Three independent implementations live here:
 
 Parity status: every function here is pinned by tests in
 ``tests/test_oracle_pins.py``, ``tests/test_oracle_mask_pins.py``,
-``tests/test_oracle_varlen_pins.py`` and
+``tests/test_oracle_varlen_pins.py``, ``tests/test_oracle_fp8_pins.py`` and
 ``tests/test_oracle_bwd_pins.py`` (closed
 forms, invariants, brute force, finite differences and the
 recurrence-equals-definition check); none is "parity unpinned".
@@ -233,6 +237,42 @@ def attention_varlen(q, k, v, cu_seqlens, scale: float | None = None, causal: bo
         O[s0:s1] = o[0].transpose(1, 0, 2)
         LSE[:, s0:s1] = lse[0]
     return O, LSE
+
+
+def decode_e4m3(codes) -> np.ndarray:
+    """fp64 values of fp8 e4m3 codes (uint8), from the format's definition:
+    bit 7 the sign, bits 6-3 the exponent e (bias 7), bits 2-0 the mantissa m;
+    e = 0 gives the subnormals m/8 * 2^-6, otherwise (1 + m/8) * 2^(e-7); the
+    one code with e = 15 and m = 7 (per sign) is NaN, and there is no
+    infinity (the "E4M3FN" variant, largest finite value 448)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where((c >> 7) & 1, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (c & 7 == 7), np.nan, mag)
+    return sign * mag
+
+
+def attention_fp8(q8, k8, v8, descale_q: float, descale_k: float, descale_v: float,
+                  scale: float | None = None, causal: bool = False, rows=None):
+    """Attention on fp8 operands in fp64: the real tensors are
+    ``descale_x * decode_e4m3(x8)``, and the result is :func:`attention` of
+    those (the FP8 inference of item 4, "低精度推理支持", of
+    "flash-attention与TensorRT 10集成", blog.gitcode.com, read as e4m3 codes
+    with one dequantisation factor per tensor).  ``q8, k8, v8``: uint8 codes
+    ``[B, H, N, d]`` (or a torch float8_e4m3fn / uint8 tensor)."""
+    def codes(x):
+        if hasattr(x, "detach"):
+            x = x.detach().cpu()
+            if x.dtype != __import__("torch").uint8:
+                x = x.view(__import__("torch").uint8)
+            x = x.numpy()
+        return np.asarray(x, dtype=np.uint8)
+    q = float(descale_q) * decode_e4m3(codes(q8))
+    k = float(descale_k) * decode_e4m3(codes(k8))
+    v = float(descale_v) * decode_e4m3(codes(v8))
+    return attention(q, k, v, scale=scale, causal=causal, rows=rows)
 
 
 def attention_bwd(q, k, v, dout, scale: float | None = None, causal: bool = False):

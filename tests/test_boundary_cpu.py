@@ -170,3 +170,23 @@ def test_python_varlen_rejects_bad_offsets_tensor():
     x = torch.zeros(8, 2, 64, dtype=torch.float16)
     with pytest.raises(ValueError):
         fa.fwd_varlen(x, x, x, torch.tensor([0, 8], dtype=torch.int64), 8)
+
+
+def test_fp8_argument_errors(lib):
+    def call(q=P, d=128, scale=0.0, dq=0.01, dk=0.01, dv=0.01, causal=0, lse=None, N=256):
+        return lib.fa_fwd_fp8(q, P, P, P, lse, 1, 2, N, d, scale, dq, dk, dv, causal, None)
+    assert call(q=None) == fa.FA_ERR_ARG
+    assert call(d=64) == fa.FA_ERR_HEADDIM
+    assert call(d=96) == fa.FA_ERR_HEADDIM
+    assert call(dq=0.0) == fa.FA_ERR_ARG
+    assert call(dk=-1.0) == fa.FA_ERR_ARG
+    assert call(dv=float("inf")) == fa.FA_ERR_ARG
+    assert call(dq=float("nan")) == fa.FA_ERR_ARG
+    assert call(scale=-0.5) == fa.FA_ERR_ARG
+    assert call(dq=1e30, dk=1e30) == fa.FA_ERR_ARG  # scale * dq * dk overflows
+    assert call(causal=3) == fa.FA_ERR_ARG
+    assert call(q=P + 4) == fa.FA_ERR_ALIGN
+    assert call(lse=P + 1) == fa.FA_ERR_ALIGN
+    # the 16-bit entry points refuse the e4m3 dtype
+    assert lib.fa_fwd(P, P, P, P, None, 1, 1, 128, 128, 0.0, 0, 2, None) == fa.FA_ERR_DTYPE
+    assert lib.fa_fwd_qkvpacked(P, P, None, 1, 128, 1, 128, 0.0, 0, 0.0, 2, None) == fa.FA_ERR_DTYPE
