@@ -222,6 +222,10 @@ int run(const Problem& pr, cudaStream_t stream) {
   if ((rc = encode_operand(&p.tmap_v, pr.v, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
                            128)) != FA_OK)
     return rc;
+  if (pr.dtype != FA_E4M3 &&
+      (rc = encode_operand(&p.tmap_o, pr.o, pr.dtype, pr.d, R, pr.H, NB, pr.osn, pr.osh, pr.osb,
+                           128)) != FA_OK)
+    return rc;
   p.o = pr.o;
   p.lse = pr.lse;
   p.o_stride_n = pr.osn;
@@ -240,6 +244,9 @@ int run(const Problem& pr, cudaStream_t stream) {
   p.alibi_slopes = pr.alibi;
   p.scale_log2 = pr.scale * pr.qk_descale * 1.4426950408889634f;
   p.o_scale = pr.v_descale;
+  // 2-byte outputs: strides are whole 128-byte rows (d >= 64), so the base decides
+  p.o_vec32 = (reinterpret_cast<uintptr_t>(pr.o) & 31u) == 0 && (pr.osn * 2) % 32 == 0 &&
+              (pr.osh * 2) % 32 == 0 && (pr.osb * 2) % 32 == 0;
   const int rows_per_tile = 128 * q_tiles_for(pr.d);
   p.num_qblocks = (pr.N + rows_per_tile - 1) / rows_per_tile;
   p.num_tiles = pr.B * pr.H * p.num_qblocks;

@@ -81,12 +81,14 @@ __device__ unsigned int g_fa_watchdog = 0u;
 enum WaitSite : unsigned {
   kSiteQEmpty = 1, kSiteKvEmpty = 2, kSiteQFull = 3, kSiteKvFull = 4, kSitePFull = 5,
   kSiteSFull = 6, kSiteODone = 7, kSiteSelfTest = 8, kSiteDrain = 9, kSiteSFree = 10,
-  kSitePFree = 11, kSiteAlign = 12, kSiteXch = 13, kSiteSeqlens = 14
+  kSitePFree = 11, kSiteAlign = 12, kSiteXch = 13, kSiteSeqlens = 14, kSiteOSlot = 15,
+  kSiteOStaged = 16
 };
 // kRoleArgs: not a wait but a device-side argument check (cu_seqlens out of
 // range); the offending work tile is skipped.
 enum Role : unsigned {
-  kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4, kRoleArgs = 5
+  kRoleProducer = 1, kRoleMma = 2, kRoleSoftmax = 3, kRoleTest = 4, kRoleArgs = 5,
+  kRoleStore = 6
 };
 
 struct FwdParams {
@@ -96,6 +98,7 @@ struct FwdParams {
   CUtensorMap tmap_q;
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
+  CUtensorMap tmap_o;  // the same view of o (16-bit outputs), for the TMA stores
   void* o;
   float* lse;  // nullptr, or indexed [bc * lse_stride_b + h * lse_stride_h + token row]
   long long o_stride_b, o_stride_h, o_stride_n;  // in elements
@@ -111,6 +114,7 @@ struct FwdParams {
   const float* alibi_slopes;  // [H]: the scaled score gets -slope[h] * |i - j|; or nullptr
   float scale_log2;  // scale * log2(e) (e4m3: times the q and k descale factors)
   float o_scale;     // factor on O / l: 1, or the v descale factor (e4m3)
+  int o_vec32;       // o and its strides are 32-byte aligned: 32-byte stores
   int num_qblocks;   // query blocks per (b, h) (of the longest sequence)
   int num_tiles;     // B * H * num_qblocks
   unsigned long long wait_limit_ns;
@@ -159,6 +163,10 @@ struct FwdCfg {
   static constexpr int PRODUCER_WARP = SOFTMAX_WARPS;
   static constexpr int MMA_S_WARP = SOFTMAX_WARPS + 1;   // issues S = Q K^T, owns TMEM
   static constexpr int MMA_PV_WARP = SOFTMAX_WARPS + 2;  // issues O += P V
+  static constexpr int STORE_WARP = SOFTMAX_WARPS + 3;   // TMA stores of O (16-bit outputs)
+  // 16-bit outputs leave the SM by TMA stores from a K/V ring slot; the e4m3
+  // path writes bf16 O, twice its slot, with per-thread stores
+  static constexpr bool O_TMA = ELT != kE4M3;
   // whole warpgroups: the softmax groups, then one group holding the producer
   // warp, the two MMA warps and one warp without a role
   static constexpr int THREADS = 128 * (SOFTMAX_WGS + 1);
@@ -172,16 +180,27 @@ struct FwdCfg {
   static constexpr int SP_OFF = QS * TILE_BYTES;
   static constexpr int SKV_OFF = SP_OFF + P_TILE_BYTES;
   static constexpr int BAR_OFF = SKV_OFF + KVS * TILE_BYTES;
-  // barrier indices ([Q tile] unless noted)
-  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_KV_FULL = 2, B_KV_EMPTY = 2 + KVS,
-                       B_S_FULL = 2 + 2 * KVS, B_S_FREE = B_S_FULL + 2,
+  // barrier indices ([Q tile] unless noted).  A ring slot holds K, V or O
+  // tiles in turn; its "full" barrier is split by consumer -- K loads complete
+  // on B_K_FULL (the S thread), V loads on B_V_FULL (the P V thread), O
+  // reservations on B_O_READY (the softmax groups) -- so every barrier has
+  // one consumer that waits each of its phases in order.  (A parity wait only
+  // tells a phase from the one before it: a shared barrier could be two
+  // phases away from a consumer that skips the others' uses.)
+  static constexpr int B_Q_FULL = 0, B_Q_EMPTY = 1, B_K_FULL = 2, B_V_FULL = 2 + KVS,
+                       B_O_READY = 2 + 2 * KVS, B_KV_EMPTY = 2 + 3 * KVS,
+                       B_S_FULL = 2 + 4 * KVS, B_S_FREE = B_S_FULL + 2,
                        B_P_FULL = B_S_FREE + 2,  // [half of P] of the tile using the buffer
                        B_P_FREE = B_P_FULL + 2,  // [Q tile][half]: that half is this tile's turn
                        B_PV_DONE = B_P_FREE + 4,  // [Q tile]: a P V product of the tile finished
                        B_O_FINAL = B_PV_DONE + 2,
                        B_XCH = B_O_FINAL + 2,  // the two softmax groups of a tile met
                        B_DRAIN = B_XCH + 2,    // [MMA thread]
-                       NUM_BARS = B_DRAIN + 2;
+                       // [ring slot]: a tile's O written into that slot.  One per slot,
+                       // so that a slot's next O use -- which needs this one's release
+                       // by the store warp -- cannot run a phase ahead of its waiter.
+                       B_O_STAGED = B_DRAIN + 2,
+                       NUM_BARS = B_O_STAGED + KVS;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int XCH_OFF = MISC_OFF + 16;  // row max / row sum exchange [tile][half][row]
   static constexpr int END_OFF = XCH_OFF + 2 * 2 * 128 * 4;
@@ -294,6 +313,22 @@ __device__ __forceinline__ int next_p_user(int s, int j, const TileInfo& ti) {
   return -1;
 }
 
+// O of Q tile s leaves through a K/V ring slot (staged by the softmax groups,
+// stored by TMA) when the output is 16-bit, the tile is not empty and -- for
+// packed variable-length sequences, where a box past the sequence's end would
+// write the next sequence's rows -- the whole 128-row box lies inside the
+// sequence.  Such tiles take one ring position each after the work tile's
+// last V: position 2 n_u for the first, 2 n_u + 1 for the second.
+template <bool O_TMA>
+__device__ __forceinline__ bool o_via_slot(const FwdParams& p, const TileInfo& ti, int s) {
+  if (!O_TMA || ti.lo[s] == ti.hi[s]) return false;
+  return p.cu_seqlens == nullptr || ti.q0 + (s + 1) * BM <= ti.len;
+}
+template <bool O_TMA>
+__device__ __forceinline__ int o_slots(const FwdParams& p, const TileInfo& ti) {
+  return (o_via_slot<O_TMA>(p, ti, 0) ? 1 : 0) + (o_via_slot<O_TMA>(p, ti, 1) ? 1 : 0);
+}
+
 // Static persistent schedule: round r hands tiles [r*G, (r+1)*G) to the G
 // CTAs, reversing the order on odd rounds, so that with the longest-first
 // causal order every CTA gets a long and a short tile in each pair of rounds.
@@ -333,18 +368,41 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0, q_count = 0;
   bool ok = true;
+  // For the drain after an abort: the last load into each slot (its barrier
+  // and the parity of the phase it completes).
+  uint32_t k_par = 0u, v_par = 0u;  // bit i: parity of slot i's next K / V load
+  uint32_t last_bar[KVS], last_par[KVS];
+#pragma unroll
+  for (int i = 0; i < KVS; ++i) last_bar[i] = 0u, last_par[i] = 0u;
   // one K or V tile into the next ring slot
-  auto load_kv = [&](const CUtensorMap* map, int row0, const TileInfo& ti) -> bool {
+  auto load_kv = [&](const CUtensorMap* map, int row0, const TileInfo& ti, bool is_k) -> bool {
     const int slot = kv_count % KVS, use = kv_count / KVS;
     if (use > 0 && !wait_phase(bars + 8 * (C::B_KV_EMPTY + slot), (use - 1) & 1, abort_flag,
                                p.wait_limit_ns, (kRoleProducer << 8) | kSiteKvEmpty))
       return false;
-    const uint32_t full = bars + 8 * (C::B_KV_FULL + slot);
+    const uint32_t full = bars + 8 * ((is_k ? C::B_K_FULL : C::B_V_FULL) + slot);
+    uint32_t& par = is_k ? k_par : v_par;
+    last_bar[slot] = full;
+    last_par[slot] = (par >> slot) & 1u;
+    par ^= 1u << slot;
     mbar_arrive_expect_tx(full, C::TILE_BYTES);
 #pragma unroll
     for (int c = 0; c < C::CHUNKS; ++c)
       tma_load_4d(base + C::SKV_OFF + slot * C::TILE_BYTES + c * C::CHUNK_BYTES, map, full,
                   c * C::BOX, ti.row0 + row0, ti.h, ti.bc);
+    ++kv_count;
+    return true;
+  };
+  // A ring position that carries O instead of a load: once the slot's previous
+  // use is released, complete its full phase without bytes, which hands the
+  // slot to the softmax groups of the tile (and keeps every slot's phases
+  // one per position).
+  auto reserve_slot = [&]() -> bool {
+    const int slot = kv_count % KVS, use = kv_count / KVS;
+    if (use > 0 && !wait_phase(bars + 8 * (C::B_KV_EMPTY + slot), (use - 1) & 1, abort_flag,
+                               p.wait_limit_ns, (kRoleProducer << 8) | kSiteKvEmpty))
+      return false;
+    mbar_arrive(bars + 8 * (C::B_O_READY + slot));
     ++kv_count;
     return true;
   };
@@ -355,7 +413,7 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
     if (ti.n_u == 0) continue;
     // The first K tile needs only a ring slot: request it before waiting for
     // the previous work tile to release the Q buffer, so the two loads overlap.
-    if (!(ok = load_kv(&p.tmap_k, ti.lo_u * BN, ti))) break;
+    if (!(ok = load_kv(&p.tmap_k, ti.lo_u * BN, ti, true))) break;
     if (q_count > 0) {
       ok = wait_phase(bars + 8 * C::B_Q_EMPTY, (q_count - 1) & 1, abort_flag, p.wait_limit_ns,
                       (kRoleProducer << 8) | kSiteQEmpty);
@@ -371,9 +429,12 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
     ++q_count;
     for (int jj = 0; ok && jj < ti.n_u; ++jj) {
       const int j = ti.lo_u + jj;
-      if (jj + 1 < ti.n_u && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti))) break;
-      ok = load_kv(&p.tmap_v, j * BN, ti);
+      if (jj + 1 < ti.n_u && !(ok = load_kv(&p.tmap_k, (j + 1) * BN, ti, true))) break;
+      ok = load_kv(&p.tmap_v, j * BN, ti, false);
     }
+#pragma unroll 1
+    for (int s = 0; ok && s < QS; ++s)
+      if (o_via_slot<C::O_TMA>(p, ti, s)) ok = reserve_slot();
   }
   if (!ok) {
     // Let the loads already issued land before the CTA's shared memory goes away.
@@ -382,11 +443,12 @@ __device__ void producer_role(const FwdParams& p, uint32_t base, volatile int* a
     if (q_count > 0)
       wait_phase(bars + 8 * C::B_Q_FULL, (q_count - 1) & 1, &no_abort_q, drain,
                  (kRoleProducer << 8) | kSiteDrain);
-    for (int i = max(0, kv_count - KVS); i < kv_count; ++i) {
+    // earlier loads into a slot landed before the slot was reused
+#pragma unroll 1
+    for (int i = 0; i < KVS; ++i) {
       volatile int no_abort = 0;
-      const uint32_t bar = bars + 8 * (C::B_KV_FULL + i % KVS);
-      if (!mbar_try_wait(bar, (i / KVS) & 1))
-        wait_phase(bar, (i / KVS) & 1, &no_abort, drain, (kRoleProducer << 8) | kSiteDrain);
+      if (last_bar[i] != 0u && !mbar_try_wait(last_bar[i], last_par[i]))
+        wait_phase(last_bar[i], last_par[i], &no_abort, drain, (kRoleProducer << 8) | kSiteDrain);
     }
   }
 }
@@ -413,9 +475,12 @@ __device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   int s_issued[2] = {0, 0};
   bool ok = true;
 
+  uint32_t k_par = 0u;  // bit i: parity of slot i's next K load
   auto wait_kv = [&](int idx) -> bool {
-    const bool r = wait_phase(bars + 8 * (C::B_KV_FULL + idx % KVS), (idx / KVS) & 1, abort_flag,
+    const int slot = idx % KVS;
+    const bool r = wait_phase(bars + 8 * (C::B_K_FULL + slot), (k_par >> slot) & 1u, abort_flag,
                               lim, (kRoleMma << 8) | kSiteKvFull);
+    k_par ^= 1u << slot;
     tc_fence_after_sync();
     return r;
   };
@@ -468,7 +533,7 @@ __device__ void mma_s_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       tc_commit(bars + 8 * (C::B_KV_EMPTY + k_idx % KVS));
       if (jj + 1 == ti.n_u) tc_commit(bars + 8 * C::B_Q_EMPTY);
     }
-    kv_count = kv0 + 2 * ti.n_u;
+    kv_count = kv0 + 2 * ti.n_u + o_slots<C::O_TMA>(p, ti);
   }
   if (!ok) {
     // Wait for every MMA this thread issued before TMEM is released.
@@ -492,7 +557,7 @@ __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const unsigned long long lim = p.wait_limit_ns;
   const int G = gridDim.x, cta = blockIdx.x;
   int kv_count = 0;
-  uint32_t p_par = 0u;
+  uint32_t p_par = 0u, v_par = 0u;  // v_par bit i: parity of slot i's next V load
   bool ok = true;
   const uint32_t pa = sw128_desc_lo(base + C::SP_OFF, 16);
 
@@ -539,8 +604,9 @@ __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     for (int jj = 0; ok && jj < ti.n_u; ++jj) {
       const int j = ti.lo_u + jj;
       const int v_idx = kv0 + ring_v(jj, ti.n_u);
-      ok = wait_phase(bars + 8 * (C::B_KV_FULL + v_idx % KVS), (v_idx / KVS) & 1, abort_flag, lim,
-                      (kRoleMma << 8) | kSiteKvFull);
+      ok = wait_phase(bars + 8 * (C::B_V_FULL + v_idx % KVS), (v_par >> (v_idx % KVS)) & 1u,
+                      abort_flag, lim, (kRoleMma << 8) | kSiteKvFull);
+      v_par ^= 1u << (v_idx % KVS);
       tc_fence_after_sync();
 #pragma unroll 1
       for (int s = 0; s < QS; ++s) {
@@ -554,7 +620,7 @@ __device__ void mma_pv_role(const FwdParams& p, uint32_t base, uint32_t tmem,
       if (!ok) break;
       tc_commit(bars + 8 * (C::B_KV_EMPTY + v_idx % KVS));
     }
-    kv_count = kv0 + 2 * ti.n_u;
+    kv_count = kv0 + 2 * ti.n_u + o_slots<C::O_TMA>(p, ti);
   }
   if (!ok) {
     volatile int no_abort = 0;
@@ -692,6 +758,8 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
   const int G = gridDim.x, cta = blockIdx.x;
   uint32_t s_par = 0u, pf_par = 0u, fin_par = 0u, x_par = 0u;
   int pv_count = 0;  // P V products of this Q tile issued before the current block
+  int kv_count = 0;  // ring positions of the work tiles so far (for the O slots)
+  uint32_t o_par = 0u;  // bit i: parity of slot i's next O reservation (both tiles' O)
   // The P buffer's first use in the kernel (tile 0, first block) has nothing
   // to wait for; every later use waits for the buffer to be handed over.
   bool first_use = s == 0;
@@ -710,6 +778,24 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const int t = tile_of(round, cta, G);
     if (t >= p.num_tiles) continue;
     const TileInfo ti = decode_tile<QS>(p, t);
+    // ring slot of this tile's O and the parity of its reservation; every
+    // group follows the reservations of both tiles
+    int o_slot = -1;
+    uint32_t o_wait_par = 0u;
+    if (ti.n_u > 0) {
+      int k = 0;
+#pragma unroll 1
+      for (int s2 = 0; s2 < QS; ++s2) {
+        if (!o_via_slot<C::O_TMA>(p, ti, s2)) continue;
+        const int slot = (kv_count + 2 * ti.n_u + k++) % KVS;
+        if (s2 == s) {
+          o_slot = slot;
+          o_wait_par = (o_par >> slot) & 1u;
+        }
+        o_par ^= 1u << slot;
+      }
+      kv_count += 2 * ti.n_u + k;
+    }
     const int lo = ti.lo[s], hi = ti.hi[s];
     if (lo == hi) continue;
     const int r_first = ti.q0 + s * BM, r_last = r_first + BM - 1;
@@ -856,6 +942,36 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     const float inv_l = p.o_scale / l_row;
     const long long trow = static_cast<long long>(ti.row0) + row;  // tensor row
     const bool store = row < ti.len && trow < p.rows_total;
+    if (o_slot >= 0) {
+      // Stage this group's columns of O in the tile's ring slot, in the
+      // 128-byte swizzled layout of the TMA box (row r's 16-byte unit u at
+      // u ^ (r % 8) of its line), for the store warp to write out by TMA.
+      const int slot = o_slot;
+      bool ok = wait_phase(bars + 8 * (C::B_O_READY + slot), o_wait_par, abort_flag, lim,
+                           (kRoleSoftmax << 8) | kSiteOSlot);
+      if (!__all_sync(0xffffffffu, ok)) return;
+      const uint32_t sbase = base + C::SKV_OFF + slot * C::TILE_BYTES + r * 128;
+#pragma unroll 1
+      for (int c = 0; c < HD2; c += 32) {
+        uint32_t ov[32];
+        tmem_ld32_sync(lane_base + o_col + c, ov);
+        uint32_t wp[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          wp[i] = pack2<OUT_BF16>(__uint_as_float(ov[2 * i]) * inv_l,
+                                  __uint_as_float(ov[2 * i + 1]) * inv_l);
+        const int col = HD2 * hf + c;  // first of these 32 columns
+        const uint32_t line = sbase + (col / 64) * C::CHUNK_BYTES;
+        const uint32_t u0 = (col % 64) / 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          st_shared_v4(line + (((u0 + i) ^ (static_cast<uint32_t>(r) & 7u)) << 4), wp[4 * i],
+                       wp[4 * i + 1], wp[4 * i + 2], wp[4 * i + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (C::B_O_STAGED + slot));
+    } else {
     T* orow = reinterpret_cast<T*>(p.o) + ti.bc * p.o_stride_b + ti.h * p.o_stride_h +
               trow * p.o_stride_n + HD2 * hf;
 #pragma unroll 1
@@ -869,10 +985,17 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
         wp[i] = pack2<OUT_BF16>(__uint_as_float(ov[2 * i]) * inv_l,
                                 __uint_as_float(ov[2 * i + 1]) * inv_l);
       if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c);
+        if (p.o_vec32) {
+          // 32-byte stores: every store fills whole 32-byte sectors
+          st_global_v8(orow + c, wp);
+          st_global_v8(orow + c + 16, wp + 8);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = w[i];
+          for (int i = 0; i < 4; ++i) dst[i] = w[i];
+        }
       }
+    }
     }
     if (hf == 0 && p.lse != nullptr && store)
       p.lse[ti.bc * p.lse_stride_b + ti.h * p.lse_stride_h + trow] =
@@ -881,6 +1004,48 @@ __device__ void softmax_role(const FwdParams& p, uint32_t base, uint32_t tmem,
     // P arrival, which comes after these loads completed.
     tc_fence_before_sync();
   }
+}
+
+// Store warp (one thread): for every Q tile whose O goes through a ring slot,
+// waits until both softmax groups have staged their columns there, writes the
+// tile out with TMA stores, waits until the stores have read the slot and
+// releases it to the producer.
+template <int HD, int QS, int KVS, int ELT>
+__device__ void store_role(const FwdParams& p, uint32_t base, volatile int* abort_flag) {
+  using C = FwdCfg<HD, QS, KVS, ELT>;
+  const uint32_t bars = base + C::BAR_OFF;
+  const int G = gridDim.x, cta = blockIdx.x;
+  int kv_count = 0;
+  uint32_t staged_par = 0u;  // bit i: parity of ring slot i's next staging
+  bool ok = true;
+  for (int round = 0; ok && round * G < p.num_tiles; ++round) {
+    const int t = tile_of(round, cta, G);
+    if (t >= p.num_tiles) continue;
+    const TileInfo ti = decode_tile<QS>(p, t);
+    if (ti.n_u == 0) continue;
+    const int kv0 = kv_count;
+    kv_count += 2 * ti.n_u + o_slots<C::O_TMA>(p, ti);
+    int k = 0;
+#pragma unroll 1
+    for (int s = 0; s < QS; ++s) {
+      if (!o_via_slot<C::O_TMA>(p, ti, s)) continue;
+      const int slot = (kv0 + 2 * ti.n_u + k++) % KVS;
+      ok = wait_phase(bars + 8 * (C::B_O_STAGED + slot), (staged_par >> slot) & 1u, abort_flag,
+                      p.wait_limit_ns, (kRoleStore << 8) | kSiteOStaged);
+      staged_par ^= 1u << slot;
+      if (!ok) break;
+      const uint32_t src = base + C::SKV_OFF + slot * C::TILE_BYTES;
+#pragma unroll
+      for (int c = 0; c < C::CHUNKS; ++c)
+        tma_store_4d(&p.tmap_o, src + c * C::CHUNK_BYTES, c * C::BOX, ti.row0 + ti.q0 + s * BM,
+                     ti.h, ti.bc);
+      bulk_commit_group();
+      bulk_wait_read_all();
+      mbar_arrive(bars + 8 * (C::B_KV_EMPTY + slot));
+    }
+  }
+  // the writes themselves complete before the CTA ends
+  bulk_wait_all();
 }
 
 template <int HD, int QS, int KVS, int ELT, bool ALIBI>
@@ -905,7 +1070,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, ELT>::THREADS, 1)
     mbar_init(bars + 8 * C::B_Q_FULL, 1);
     mbar_init(bars + 8 * C::B_Q_EMPTY, 1);
     for (int i = 0; i < KVS; ++i) {
-      mbar_init(bars + 8 * (C::B_KV_FULL + i), 1);
+      mbar_init(bars + 8 * (C::B_K_FULL + i), 1);
+      mbar_init(bars + 8 * (C::B_V_FULL + i), 1);
+      mbar_init(bars + 8 * (C::B_O_READY + i), 1);
       mbar_init(bars + 8 * (C::B_KV_EMPTY + i), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -918,6 +1085,8 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, ELT>::THREADS, 1)
       mbar_init(bars + 8 * (C::B_O_FINAL + i), 1);
       mbar_init(bars + 8 * (C::B_DRAIN + i), 1);
     }
+    for (int i = 0; i < KVS; ++i)
+      mbar_init(bars + 8 * (C::B_O_STAGED + i), 8);  // one arrival per softmax warp of the tile
     // first P half: the first group's warps once P is written and the second
     // group's once their O half is rescaled; second half: the second group
     mbar_init(bars + 8 * C::B_P_FULL, 8);
@@ -929,6 +1098,7 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, ELT>::THREADS, 1)
     tma_prefetch_desc(&p.tmap_q);
     tma_prefetch_desc(&p.tmap_k);
     tma_prefetch_desc(&p.tmap_v);
+    if (C::O_TMA) tma_prefetch_desc(&p.tmap_o);
   }
   if (warp == C::MMA_S_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -954,7 +1124,9 @@ __global__ void __launch_bounds__(FwdCfg<HD, QS, KVS, ELT>::THREADS, 1)
     if (lane == 0) mma_s_role<HD, QS, KVS, ELT>(p, base, tmem, abort_flag);
   } else if (warp == C::MMA_PV_WARP) {
     if (lane == 0) mma_pv_role<HD, QS, KVS, ELT>(p, base, tmem, abort_flag);
-  }  // the last warp has no role
+  } else if (warp == C::STORE_WARP) {
+    if (lane == 0 && C::O_TMA) store_role<HD, QS, KVS, ELT>(p, base, abort_flag);
+  }
 
   tc_fence_before_sync();
   __syncthreads();
