@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/fa.h"
@@ -22,6 +23,8 @@ constexpr int kVersion = 1 * 10000 + 2 * 100 + 0;  // 1.2.0: local window, ALiBi
 #define FA_WAIT_LIMIT_NS 2000000000ull
 #endif
 constexpr unsigned long long kWaitLimitNs = FA_WAIT_LIMIT_NS;
+// Bound of every mbarrier wait of the next launches (fa_debug_set_wait_limit).
+std::atomic<unsigned long long> g_wait_limit_ns{kWaitLimitNs};
 constexpr int kMaxDevices = 64;
 
 // Row-statistic scratch of fa_bwd_noalloc: a library-owned device array, one
@@ -250,7 +253,7 @@ int run(const Problem& pr, cudaStream_t stream) {
   const int rows_per_tile = 128 * q_tiles_for(pr.d);
   p.num_qblocks = (pr.N + rows_per_tile - 1) / rows_per_tile;
   p.num_tiles = pr.B * pr.H * p.num_qblocks;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = g_wait_limit_ns.load();
 
   const bool alibi = pr.alibi != nullptr;
   switch (pr.d) {
@@ -488,7 +491,7 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const fl
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.nblk = (N + 127) / 128;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = g_wait_limit_ns.load();
   const bool bf16 = dtype == FA_BF16;
   if (d == 64) return bf16 ? launch_bwd<64, true>(p, *st, s) : launch_bwd<64, false>(p, *st, s);
   return bf16 ? launch_bwd<128, true>(p, *st, s) : launch_bwd<128, false>(p, *st, s);
@@ -561,6 +564,12 @@ int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st* 
   if (limit_ns == 0 || limit_ns > 10000000000ull) return FA_ERR_ARG;
   watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_ns);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_debug_set_wait_limit(unsigned long long limit_ns) {
+  if (limit_ns != 0 && (limit_ns < 100 || limit_ns > 10000000000ull)) return FA_ERR_ARG;
+  g_wait_limit_ns.store(limit_ns == 0 ? kWaitLimitNs : limit_ns);
+  return FA_OK;
 }
 
 int fa_debug_exp2_poly(const float* x, float* y, int n, struct CUstream_st* stream) {

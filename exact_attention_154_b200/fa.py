@@ -45,6 +45,7 @@ SIGNATURES = {
     "fa_debug_watchdog_selftest": (_I, [ctypes.c_ulonglong, _VP]),
     "fa_launch_ctas": (_I, [_I, _I, _I, _I, _I]),
     "fa_debug_exp2_poly": (_I, [_VP, _VP, _I, _VP]),
+    "fa_debug_set_wait_limit": (_I, [ctypes.c_ulonglong]),
     "fa_version": (_I, []),
 }
 
@@ -350,6 +351,14 @@ def watchdog_selftest(limit_ns: int = 20_000_000):
                                            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     if rc != FA_OK:
         raise FaError(rc, "fa_debug_watchdog_selftest")
+
+
+def set_wait_limit(limit_ns: int = 0):
+    """Bound (ns) of every mbarrier wait in the kernels launched next; 0
+    restores the default.  A debug hook for testing the kernels' give-up path."""
+    rc = load().fa_debug_set_wait_limit(int(limit_ns))
+    if rc != FA_OK:
+        raise FaError(rc, "fa_debug_set_wait_limit")
 
 
 def exp2_poly(x: torch.Tensor) -> torch.Tensor:

@@ -250,6 +250,19 @@ int fa_device_status(int clear, unsigned int *detail);
 int fa_debug_watchdog_selftest(unsigned long long limit_ns, struct CUstream_st *stream);
 
 /*
+ * Debug: bound of every mbarrier wait inside the attention kernels launched
+ * after this call, in nanoseconds (100 ns .. 10 s; 0 restores the default of
+ * 2 s).  With a bound far below a tile's load or product time, the kernels'
+ * waits run out: each CTA raises its abort flag, drains the loads and products
+ * it issued, frees tensor memory and returns, and fa_device_status() reports
+ * FA_ERR_TIMEOUT with the (role << 8) | site of the first wait that gave up.
+ * For testing that failure path on the real kernels; outputs of such launches
+ * are undefined.  Applies to every device and thread of the process.
+ * Returns FA_OK or FA_ERR_ARG.
+ */
+int fa_debug_set_wait_limit(unsigned long long limit_ns);
+
+/*
  * Test hook: y[i] = the kernel's software 2^x (the FMA-pipe exponential used
  * for a quarter of the softmax weights at head dim 256) for n device floats x.  Not part of the
  * attention method; exposed so that its error against exp2f can be measured.

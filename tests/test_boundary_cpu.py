@@ -190,3 +190,9 @@ def test_fp8_argument_errors(lib):
     # the 16-bit entry points refuse the e4m3 dtype
     assert lib.fa_fwd(P, P, P, P, None, 1, 1, 128, 128, 0.0, 0, 2, None) == fa.FA_ERR_DTYPE
     assert lib.fa_fwd_qkvpacked(P, P, None, 1, 128, 1, 128, 0.0, 0, 0.0, 2, None) == fa.FA_ERR_DTYPE
+
+
+def test_wait_limit_hook_argument_check(lib):
+    assert lib.fa_debug_set_wait_limit(50) == fa.FA_ERR_ARG
+    assert lib.fa_debug_set_wait_limit(10**11) == fa.FA_ERR_ARG
+    assert lib.fa_debug_set_wait_limit(0) == fa.FA_OK  # the default
