@@ -269,12 +269,15 @@ def time_device(go, steps, warmup, world):
     stream = torch.cuda.current_stream()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
+    t0 = time.perf_counter()
     for _ in range(steps):
         go()
+    host_ms = (time.perf_counter() - t0) * 1e3 / steps
     end.record(stream)
     torch.cuda.synchronize()
     dist_barrier(world)
     ms = start.elapsed_time(end) / steps
+    time_device.host_ms = host_ms  # enqueue time per step (Python + C ABI + launch)
     return dist_max(ms, world)
 
 
@@ -467,6 +470,7 @@ def bench_gpu(args, w, key, world, rank, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4), "steps": e2e_steps},
         "gpu_launches": steps,
+        "host_ms_per_step": round(time_device.host_ms, 5),
         "clocks": clocks,
     }
     if not clocks_ok(clocks):

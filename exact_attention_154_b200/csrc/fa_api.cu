@@ -38,20 +38,25 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// g_mutex guards only first-time set-up (the driver entry point, a device's
+// attributes, a kernel's shared-memory attribute, the scratch address); the
+// steady-state call path takes no lock.
 std::mutex g_mutex;
-EncodeTiledFn g_encode = nullptr;
+std::atomic<EncodeTiledFn> g_encode{nullptr};
 struct DeviceState {
-  bool ready = false;
+  std::atomic<bool> ready{false};
   bool is_sm100 = false;
   int sm_count = 0;
-  bool attr_set[18] = {};
-  bool bwd_attr_set[8] = {false, false, false, false, false, false, false, false};
-  float* bwd_scratch = nullptr;  // this device's g_bwd_scratch
+  std::atomic<bool> attr_set[18] = {};
+  std::atomic<bool> bwd_attr_set[8] = {};
+  std::atomic<float*> bwd_scratch{nullptr};  // this device's g_bwd_scratch
 };
 DeviceState g_dev[kMaxDevices];
 
 int get_encode_fn() {
-  if (g_encode) return FA_OK;
+  if (g_encode.load(std::memory_order_acquire)) return FA_OK;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_encode.load(std::memory_order_relaxed)) return FA_OK;
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
   if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
@@ -60,7 +65,7 @@ int get_encode_fn() {
     cudaGetLastError();
     return FA_ERR_CUDA;
   }
-  g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  g_encode.store(reinterpret_cast<EncodeTiledFn>(fn), std::memory_order_release);
   return FA_OK;
 }
 
@@ -71,21 +76,39 @@ int device_state(DeviceState** out, int* dev_out) {
     return FA_ERR_CUDA;
   }
   DeviceState& st = g_dev[dev];
-  if (!st.ready) {
-    int major = 0, minor = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_CUDA;
+  if (!st.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!st.ready.load(std::memory_order_relaxed)) {
+      int major = 0, minor = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+      }
+      st.is_sm100 = (major == 10 && minor == 0);
+      st.sm_count = sms;
+      st.ready.store(true, std::memory_order_release);
     }
-    st.is_sm100 = (major == 10 && minor == 0);
-    st.sm_count = sms;
-    st.ready = true;
   }
   if (!st.is_sm100) return FA_ERR_DEVICE;
   *out = &st;
   *dev_out = dev;
+  return FA_OK;
+}
+
+// Sets a kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+int ensure_smem_attr(std::atomic<bool>& flag, Kernel kernel, int bytes) {
+  if (flag.load(std::memory_order_acquire)) return FA_OK;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (flag.load(std::memory_order_relaxed)) return FA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  flag.store(true, std::memory_order_release);
   return FA_OK;
 }
 
@@ -102,10 +125,48 @@ int encode_operand(CUtensorMap* map, const void* ptr, int dtype, int d, int N, i
   const CUtensorMapDataType t = dtype == FA_E4M3   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                 : dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUresult r = g_encode(map, t, 4, const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = g_encode.load(std::memory_order_acquire)(
+      map, t, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Tensor maps depend only on these arguments, so a thread keeps the last few
+// it encoded: a repeated call on the same buffers skips the encoding.
+struct MapKey {
+  const void* ptr;
+  long long sn, sh, sb;
+  int dtype, d, N, H, B, rows;
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+constexpr int kMapCache = 16;
+thread_local MapEntry t_maps[kMapCache];
+thread_local int t_next_map = 0;
+
+int encode_cached(CUtensorMap* map, const void* ptr, int dtype, int d, int N, int H, int B,
+                  long long sn, long long sh, long long sb, int rows) {
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));  // padding compares equal
+  key.ptr = ptr; key.sn = sn; key.sh = sh; key.sb = sb;
+  key.dtype = dtype; key.d = d; key.N = N; key.H = H; key.B = B; key.rows = rows;
+  for (int i = 0; i < kMapCache; ++i)
+    if (t_maps[i].valid && std::memcmp(&t_maps[i].key, &key, sizeof(key)) == 0) {
+      *map = t_maps[i].map;
+      return FA_OK;
+    }
+  const int rc = encode_operand(map, ptr, dtype, d, N, H, B, sn, sh, sb, rows);
+  if (rc != FA_OK) return rc;
+  MapEntry& e = t_maps[t_next_map];
+  t_next_map = (t_next_map + 1) % kMapCache;
+  e.key = key;
+  e.map = *map;
+  e.valid = true;
+  return FA_OK;
 }
 
 // Kernel configuration per head dim and element size: (Q tiles per work
@@ -128,14 +189,8 @@ int launch(FwdParams& p, DeviceState& st, cudaStream_t stream) {
   using C = FwdCfg<HD, QS, KVS, ELT>;
   auto kernel = fa_fwd_kernel<HD, QS, KVS, ELT, ALIBI>;
   const int slot = ((HD == 64 ? 0 : HD == 128 ? 1 : 2) * 3 + ELT) * 2 + (ALIBI ? 1 : 0);
-  if (!st.attr_set[slot]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_CUDA;
-    }
-    st.attr_set[slot] = true;
-  }
+  const int rc = ensure_smem_attr(st.attr_set[slot], kernel, C::SMEM_BYTES);
+  if (rc != FA_OK) return rc;
   const int grid = p.num_tiles < st.sm_count ? p.num_tiles : st.sm_count;
   kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -206,7 +261,6 @@ int launch_elt(FwdParams& p, int dtype, bool alibi, DeviceState& st, cudaStream_
 }
 
 int run(const Problem& pr, cudaStream_t stream) {
-  std::lock_guard<std::mutex> lock(g_mutex);
   int rc = get_encode_fn();
   if (rc != FA_OK) return rc;
   DeviceState* st = nullptr;
@@ -216,17 +270,17 @@ int run(const Problem& pr, cudaStream_t stream) {
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
   const int R = pr.map_rows, NB = pr.map_batches;
-  if ((rc = encode_operand(&p.tmap_q, pr.q, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
+  if ((rc = encode_cached(&p.tmap_q, pr.q, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
                            128)) != FA_OK)
     return rc;
-  if ((rc = encode_operand(&p.tmap_k, pr.k, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
+  if ((rc = encode_cached(&p.tmap_k, pr.k, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
                            128)) != FA_OK)
     return rc;
-  if ((rc = encode_operand(&p.tmap_v, pr.v, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
+  if ((rc = encode_cached(&p.tmap_v, pr.v, pr.dtype, pr.d, R, pr.H, NB, pr.sn, pr.sh, pr.sb,
                            128)) != FA_OK)
     return rc;
   if (pr.dtype != FA_E4M3 &&
-      (rc = encode_operand(&p.tmap_o, pr.o, pr.dtype, pr.d, R, pr.H, NB, pr.osn, pr.osh, pr.osb,
+      (rc = encode_cached(&p.tmap_o, pr.o, pr.dtype, pr.d, R, pr.H, NB, pr.osn, pr.osh, pr.osb,
                            128)) != FA_OK)
     return rc;
   p.o = pr.o;
@@ -305,14 +359,8 @@ int launch_bwd_kernel(const BwdParams& p, DeviceState& st, cudaStream_t stream) 
   using C = BwdCfg<HD, KV>;
   auto kernel = fa_bwd_kernel<HD, BF16, KV>;
   const int slot = (HD == 64 ? 0 : 4) + (BF16 ? 2 : 0) + (KV ? 1 : 0);
-  if (!st.bwd_attr_set[slot]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_CUDA;
-    }
-    st.bwd_attr_set[slot] = true;
-  }
+  const int rc = ensure_smem_attr(st.bwd_attr_set[slot], kernel, C::SMEM_BYTES);
+  if (rc != FA_OK) return rc;
   kernel<<<p.B * p.H * p.nblk, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -453,30 +501,36 @@ int check_bwd(const void* q, const void* k, const void* v, const void* o, const 
 int run_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
             const void* dout, void* dq, void* dk, void* dv, float* workspace, int B, int H, int N,
             int d, float scale, int causal, int dtype, cudaStream_t s) {
-  std::lock_guard<std::mutex> lock(g_mutex);
   int rc = get_encode_fn();
   if (rc != FA_OK) return rc;
   DeviceState* st = nullptr;
   int dev = 0;
   if ((rc = device_state(&st, &dev)) != FA_OK) return rc;
   if (workspace == nullptr) {
-    if (st->bwd_scratch == nullptr) {
-      void* ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || ptr == nullptr) {
-        cudaGetLastError();
-        return FA_ERR_CUDA;
+    float* scratch = st->bwd_scratch.load(std::memory_order_acquire);
+    if (scratch == nullptr) {
+      // this device's address of the array, looked up once with the device current
+      std::lock_guard<std::mutex> lock(g_mutex);
+      scratch = st->bwd_scratch.load(std::memory_order_relaxed);
+      if (scratch == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || ptr == nullptr) {
+          cudaGetLastError();
+          return FA_ERR_CUDA;
+        }
+        scratch = static_cast<float*>(ptr);
+        st->bwd_scratch.store(scratch, std::memory_order_release);
       }
-      st->bwd_scratch = static_cast<float*>(ptr);
     }
-    workspace = st->bwd_scratch;
+    workspace = scratch;
   }
   BwdParams p;
   std::memset(&p, 0, sizeof(p));
   const long long sn = d, sh = (long long)N * d, sb = (long long)H * N * d;
-  if ((rc = encode_operand(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
-  if ((rc = encode_operand(&p.tmap_do, dout, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_cached(&p.tmap_q, q, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_cached(&p.tmap_k, k, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_cached(&p.tmap_v, v, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
+  if ((rc = encode_cached(&p.tmap_do, dout, dtype, d, N, H, B, sn, sh, sb, 128)) != FA_OK) return rc;
   p.o = o;
   p.dout = dout;
   p.lse = lse;
@@ -585,7 +639,6 @@ int fa_launch_ctas(int B, int H, int N, int d, int causal) {
   float scale = 0.f;
   int rc = check_common(B, H, N, d, &scale, causal, FA_BF16);
   if (rc != FA_OK) return rc;
-  std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState* st = nullptr;
   int dev = 0;
   if ((rc = device_state(&st, &dev)) != FA_OK) return rc;
