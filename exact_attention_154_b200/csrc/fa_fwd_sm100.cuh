@@ -165,8 +165,10 @@ struct FwdCfg {
   static constexpr int MMA_PV_WARP = SOFTMAX_WARPS + 2;  // issues O += P V
   static constexpr int STORE_WARP = SOFTMAX_WARPS + 3;   // TMA stores of O (16-bit outputs)
   // 16-bit outputs leave the SM by TMA stores from a K/V ring slot; the e4m3
-  // path writes bf16 O, twice its slot, with per-thread stores
-  static constexpr bool O_TMA = ELT != kE4M3;
+  // path writes bf16 O, twice its slot, with per-thread stores, and so does
+  // head dim 256, whose two-slot ring cannot spare a slot at a work tile's
+  // end (measured 1-2% slower with it)
+  static constexpr bool O_TMA = ELT != kE4M3 && HD != 256;
   // whole warpgroups: the softmax groups, then one group holding the producer
   // warp, the two MMA warps and one warp without a role
   static constexpr int THREADS = 128 * (SOFTMAX_WGS + 1);

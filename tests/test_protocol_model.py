@@ -17,6 +17,7 @@ CASES = [
     dict(N=2048, causal=False, QS=2, KVS=4, B=4, H=16),
     dict(N=2048, causal=True, QS=2, KVS=4, B=4, H=16),
     dict(N=8192, causal=True, QS=1, KVS=2, B=1, H=8),
+    dict(N=8192, causal=True, QS=1, KVS=2, B=1, H=8, o_tma=False),
     dict(N=777, causal=True, QS=2, KVS=10, B=2, H=3),
     dict(N=1024, causal=True, QS=2, KVS=4, B=2, H=2, left=100),
     dict(N=600, causal=True, QS=2, KVS=4, lens=[1, 7, 128, 0, 129, 300, 513, 256], H=3),
