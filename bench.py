@@ -281,11 +281,60 @@ def time_device(go, steps, warmup, world):
     return dist_max(ms, world)
 
 
+def pipelined_e2e(host, run, outs_host, steps, warmup, world, nbuf=2):
+    """End-to-end steps through the public API: every step copies its inputs
+    from pinned host memory (``host``), runs ``run(device_inputs)`` on the
+    current stream and copies the returned tensors back into ``outs_host``.
+    The copies run on their own streams against ``nbuf`` device buffer sets,
+    so step k+1's upload and step k-1's download overlap step k's compute
+    (a buffer set is reused only after its compute and download are done).
+    Returns ms per step (max over ranks), measured from the first upload to
+    the last download with CUDA events."""
+    dev = [[torch.empty_like(t, device="cuda") for t in host] for _ in range(nbuf)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]
+    ev_out = [torch.cuda.Event() for _ in range(nbuf)]
+
+    def step(i):
+        b = i % nbuf
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_done[b])  # the last compute on this set has read it
+            for h, d in zip(host, dev[b]):
+                d.copy_(h, non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])  # this set's previous outputs are downloaded
+        outs = run(dev[b])
+        ev_done[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            for o, h in zip(outs, outs_host):
+                h.copy_(o, non_blocking=True)
+                o.record_stream(s_out)
+            ev_out[b].record(s_out)
+
+    for i in range(warmup):
+        step(i)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)
+    for i in range(steps):
+        step(i)
+    s_out.wait_stream(comp)
+    end.record(s_out)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    return dist_max(start.elapsed_time(end) / steps, world)
+
+
 def time_e2e(w, steps, warmup, world):
     """Same metric through the public Python API with pinned host inputs:
-    H2D of q, k, v (or qkv), the forward, D2H of O and LSE, every step."""
+    H2D of q, k, v (or qkv), the forward, D2H of O and LSE, every step
+    (pipelined across steps, see pipelined_e2e)."""
     host = [t.pin_memory() for t in synth.make_inputs(w)]
-    dev = [torch.empty_like(t, device="cuda") for t in host]
     if w.layout == "packed":
         o_host = torch.empty((w.B, w.N, w.H, w.d), dtype=host[0].dtype).pin_memory()
     elif w.dtype == synth.E4M3:
@@ -294,39 +343,22 @@ def time_e2e(w, steps, warmup, world):
     else:
         o_host = torch.empty_like(host[0]).pin_memory()
     lse_host = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
-    stream = torch.cuda.current_stream()
     slopes = synth.alibi_slopes(w.H).cuda() if w.alibi else None
     if w.layout == "varlen":
         lse_host = torch.empty((w.H, host[0].shape[0]), dtype=torch.float32).pin_memory()
 
-    def step():
-        for h, d in zip(host, dev):
-            d.copy_(h, non_blocking=True)
+    def run(dev):
         if w.layout == "packed":
-            o, lse = fa.fwd_qkvpacked(dev[0], causal=w.causal)
-        elif w.dtype == synth.E4M3:
-            o, lse = fa.fwd_fp8(dev[0], dev[1], dev[2], *factors, causal=w.causal)
-        elif w.layout == "varlen":
-            o, lse = fa.fwd_varlen(dev[0], dev[1], dev[2], dev[3], w.N, causal=w.causal,
-                                   window_size=w.window, alibi_slopes=slopes)
-        else:
-            o, lse = fa.fwd(dev[0], dev[1], dev[2], causal=w.causal, window_size=w.window,
-                            alibi_slopes=slopes)
-        o_host.copy_(o, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
+            return fa.fwd_qkvpacked(dev[0], causal=w.causal)
+        if w.dtype == synth.E4M3:
+            return fa.fwd_fp8(dev[0], dev[1], dev[2], *factors, causal=w.causal)
+        if w.layout == "varlen":
+            return fa.fwd_varlen(dev[0], dev[1], dev[2], dev[3], w.N, causal=w.causal,
+                                 window_size=w.window, alibi_slopes=slopes)
+        return fa.fwd(dev[0], dev[1], dev[2], causal=w.causal, window_size=w.window,
+                      alibi_slopes=slopes)
 
-    for _ in range(warmup):
-        step()
-    dist_barrier(world)
-    torch.cuda.synchronize()
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for _ in range(steps):
-        step()
-    end.record(stream)
-    torch.cuda.synchronize()
-    dist_barrier(world)
-    ms = dist_max(start.elapsed_time(end) / steps, world)
+    ms = pipelined_e2e(host, run, [o_host, lse_host], steps, warmup, world)
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = o_host.numel() * o_host.element_size() + lse_host.numel() * 4
     return ms, h2d, d2h
@@ -514,27 +546,10 @@ def bench_gpu_bwd(args, w, key, world, rank, local):
     # end to end: host q, k, v, O, LSE, dO in; dQ, dK, dV out, every step
     pinned = [t.pin_memory() for t in host] + [o.cpu().pin_memory(), lse.cpu().pin_memory()]
     outs = [torch.empty_like(t).pin_memory() for t in host[:3]]
-    devs = [torch.empty_like(t, device="cuda") for t in pinned]
-
-    def step():
-        for h_, d_ in zip(pinned, devs):
-            d_.copy_(h_, non_blocking=True)
-        grads = fa.bwd(devs[0], devs[1], devs[2], devs[4], devs[5], devs[3], causal=w.causal)
-        for g_, h_ in zip(grads, outs):
-            h_.copy_(g_, non_blocking=True)
     e2e_steps = max(3, min(args.steps, 30))
-    for _ in range(3):
-        step()
-    dist_barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    dist_barrier(world)
-    e2e_ms = dist_max(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_ms = pipelined_e2e(
+        pinned, lambda d: fa.bwd(d[0], d[1], d[2], d[4], d[5], d[3], causal=w.causal), outs,
+        e2e_steps, 3, world)
     rc, detail = fa.device_status(clear=True)
     if rc != fa.FA_OK:
         raise RuntimeError(f"kernel watchdog fired ({detail:#x})")
