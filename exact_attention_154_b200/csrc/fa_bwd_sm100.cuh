@@ -16,10 +16,14 @@
 //
 // bwd_dkdv_kernel: one CTA per 128-key block j.  For every query block i it
 // computes S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM (tcgen05, SS),
-// forms P^T and dS^T in 16 bits in shared memory (one thread per key row),
-// and accumulates dV_j += P^T dO_i and dK_j += dS^T Q_i in TMEM.
+// forms P^T and dS^T in 16 bits (one thread per key row) and writes them back
+// into TMEM over the S^T / dP^T columns it has read, and accumulates
+// dV_j += P^T dO_i and dK_j += dS^T Q_i in TMEM with P^T and dS^T as TMEM
+// operands (tcgen05.mma with A in tensor memory).
 // bwd_dq_kernel: one CTA per 128-query block i; recomputes S and dP the same
 // way for every key block j and accumulates dQ_i += dS K_j in TMEM.
+// Keeping the 16-bit tiles in TMEM leaves shared memory for two slots of the
+// streamed pair in both kernels, so the next block loads during this one.
 //
 // Roles per CTA (320 threads): warps 0-7 compute P and dS (thread = TMEM
 // lane = tile row; warps 0-3 take columns 0-63 of each block, warps 4-7
@@ -57,41 +61,44 @@ struct BwdCfg {
   static constexpr int CHUNKS = HD / 64;
   static constexpr int CHUNK_BYTES = 128 * 128;
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;   // one [128 x HD] 16-bit tile
-  static constexpr int SQR_BYTES = 2 * CHUNK_BYTES;         // one [128 x 128] 16-bit tile
   // two compute warpgroups (key/query rows x 64 of the 128 columns each),
   // then the producer warp and the MMA warp
   static constexpr int COMPUTE_WARPS = 8;
   static constexpr int THREADS = 32 * (COMPUTE_WARPS + 2);
   static constexpr int PRODUCER_WARP = COMPUTE_WARPS, MMA_WARP = COMPUTE_WARPS + 1;
   // Shared memory: the resident pair (K, V for dK/dV; Q, dO for dQ), STAGES
-  // slots of the streamed pair (Q, dO / K, V), the 16-bit P^T and dS^T tiles
-  // (dK/dV) or dS tile (dQ), per-warp column statistics (dK/dV), barriers.
-  // Two streamed slots where they fit, so the next block loads while this one
-  // is computed.
+  // slots of the streamed pair (Q, dO / K, V), per-warp column statistics
+  // (dK/dV), barriers.  Two streamed slots where they fit, so the next block
+  // loads while this one is computed.
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int SQR_TILES = KV ? 2 : 1;
   static constexpr int VEC_BYTES = KV ? COMPUTE_WARPS * 2 * 64 * 4 : 0;
   static constexpr int B_RES_FULL = 0, B_STR_FULL = 1 /* [stage] */, B_STR_EMPTY = 3 /* [stage] */,
-                       B_SD_FULL = 5, B_PDS_FULL = 6, B_PDS_FREE = 7, B_DONE = 8, B_DRAIN = 9,
+                       B_SD_FULL = 5, B_PDS_FULL = 6, B_DONE = 8, B_DRAIN = 9,
                        NUM_BARS = 10;
-  static constexpr int FIXED_BYTES = 2 * TILE_BYTES + SQR_TILES * SQR_BYTES + VEC_BYTES +
+  static constexpr int FIXED_BYTES = 2 * TILE_BYTES + VEC_BYTES +
                                      NUM_BARS * 8 + 16 + 1024;
   static constexpr int STAGES = FIXED_BYTES + 2 * STAGE_BYTES <= 232448 ? 2 : 1;
   static constexpr int SA_OFF = 0;                           // K (dkdv) / Q (dq)
   static constexpr int SB_OFF = TILE_BYTES;                  // V (dkdv) / dO (dq)
   static constexpr int SSTR_OFF = 2 * TILE_BYTES;            // slot s: Q / K at +s*STAGE_BYTES,
                                                              // dO / V at +TILE_BYTES
-  static constexpr int SP_OFF = SSTR_OFF + STAGES * STAGE_BYTES;  // P^T (dkdv only)
-  static constexpr int SDS_OFF = SP_OFF + (KV ? SQR_BYTES : 0);   // dS^T (dkdv) / dS (dq)
-  static constexpr int VEC_OFF = SDS_OFF + SQR_BYTES;
+  static constexpr int VEC_OFF = SSTR_OFF + STAGES * STAGE_BYTES;
   static constexpr int BAR_OFF = VEC_OFF + VEC_BYTES;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int END_OFF = MISC_OFF + 16;
   static constexpr int SMEM_BYTES = END_OFF + 1024;  // + slack to align the base to 1024
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  // TMEM columns: S (or S^T), dP (or dP^T), then the accumulators
+  // TMEM columns: S (or S^T), dP (or dP^T), then the accumulators.  The
+  // 16-bit P (P^T) and dS (dS^T) overwrite the first half of each 64-column
+  // group's S / dP columns: columns [64 g, 64 g + 32) hold the packed values of
+  // columns [64 g, 64 g + 64) of the tile, written by compute group g.
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0_COL = 256, ACC1_COL = 256 + HD;
+  // TMEM column of the packed 16-bit operand for MMA K-step kk (16 columns
+  // of the tile, 8 packed TMEM columns)
+  __host__ __device__ static constexpr uint32_t packed_col(int kk) {
+    return 64u * static_cast<uint32_t>(kk / 4) + 8u * static_cast<uint32_t>(kk % 4);
+  }
 };
 
 // D_i = dO_i . O_i in fp32, one warp per row.
@@ -111,20 +118,6 @@ __global__ void __launch_bounds__(256) bwd_dsum_kernel(const void* __restrict__ 
 #pragma unroll
   for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
   if (lane == 0) dsum[row] = acc;
-}
-
-// 32 packed 16-bit pairs of one tile row into the 128-byte-swizzled K-major
-// layout the MMAs read (as store_p_chunk): row r of a 64-column chunk at
-// r * 128 bytes, its 16-byte group u at u ^ (r % 8).  `col0` is a multiple of
-// 32 in [0, 128): columns col0 .. col0 + 31.
-__device__ __forceinline__ void store_row32(uint32_t tile, int r, int col0, const uint32_t* pk) {
-  const uint32_t row = tile + static_cast<uint32_t>(col0 / 64) * (128u * 128u) +
-                       static_cast<uint32_t>(r) * 128u;
-  const uint32_t u0 = static_cast<uint32_t>((col0 % 64) / 8);
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-    st_shared_v4(row + (((u0 + u) ^ (static_cast<uint32_t>(r) & 7u)) << 4), pk[4 * u],
-                 pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
 }
 
 // Loads one [128 x HD] tile of a 4-D tensor map into shared memory.
@@ -243,8 +236,6 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       tc_fence_after_sync();
       // K-major [128 x HD] operands: resident A-side tiles and streamed B-side tiles
       const uint32_t a0 = sw128_desc_lo(base + C::SA_OFF, 16), a1 = sw128_desc_lo(base + C::SB_OFF, 16);
-      // 16-bit [128 x 128] tiles written by the compute warps (K-major, K = 128)
-      const uint32_t pt = sw128_desc_lo(base + C::SP_OFF, 16), dst = sw128_desc_lo(base + C::SDS_OFF, 16);
       for (int it = 0; ok && it < count; ++it) {
         const int stage = it % C::STAGES;
         const uint32_t slot = base + C::SSTR_OFF + stage * C::STAGE_BYTES;
@@ -276,24 +267,25 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
                               (kRoleMma << 8) | kSitePFull)))
           break;
         tc_fence_after_sync();
-        // the 16-bit tiles contract over their 128 columns in 8 K-steps
+        // the 16-bit tiles (in TMEM) contract over their 128 columns in 8
+        // K-steps; the next S / dP products, issued after these by this same
+        // thread, overwrite their columns only once these have read them
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ka = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
           const uint32_t kb = (kk * 16 * 128) >> 4;
           const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t pcol = C::packed_col(kk);
           if (KV) {
             // dV += P^T dO, dK += dS^T Q
-            mma_ss(tmem + C::ACC0_COL, desc_from_lo(pt + ka), desc_from_lo(md + kb), idesc_acc, acc);
-            mma_ss(tmem + C::ACC1_COL, desc_from_lo(dst + ka), desc_from_lo(mq + kb), idesc_acc, acc);
+            mma_ts(tmem + C::ACC0_COL, tmem + C::S_COL + pcol, desc_from_lo(md + kb), idesc_acc, acc);
+            mma_ts(tmem + C::ACC1_COL, tmem + C::DP_COL + pcol, desc_from_lo(mq + kb), idesc_acc, acc);
           } else {
             // dQ += dS K
-            mma_ss(tmem + C::ACC0_COL, desc_from_lo(dst + ka), desc_from_lo(mq + kb), idesc_acc, acc);
+            mma_ts(tmem + C::ACC0_COL, tmem + C::DP_COL + pcol, desc_from_lo(mq + kb), idesc_acc, acc);
           }
         }
-        // frees the streamed slot and the 16-bit tiles
+        // frees the streamed slot
         tc_commit(bars + 8 * (C::B_STR_EMPTY + stage));
-        tc_commit(bars + 8 * C::B_PDS_FREE);
       }
       if (ok) {
         tc_commit(bars + 8 * C::B_DONE);
@@ -336,13 +328,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
                       (kRoleSoftmax << 8) | kSiteSFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
-      // the 16-bit tiles of the previous step have been read
-      if (it > 0) {
-        ok = wait_phase(bars + 8 * C::B_PDS_FREE, (it - 1) & 1, abort_flag, lim,
-                        (kRoleSoftmax << 8) | kSitePFree);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after_sync();
-      }
+      // (the previous step's 16-bit tiles in TMEM were read by its products,
+      // which the MMA thread issued before this step's S / dP)
 #pragma unroll 1
       for (int c0 = cb; c0 < cb + 64; c0 += 32) {
         uint32_t sv[32], dv[32];
@@ -375,10 +362,13 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           pk[q] = pack2<BF16>(pp[0], pp[1]);
           dk[q] = pack2<BF16>(ds[0], ds[1]);
         }
-        if (KV) store_row32(base + C::SP_OFF, r, c0, pk);
-        store_row32(base + C::SDS_OFF, r, c0, dk);
+        // packed over the columns of this group already read: 32 tile
+        // columns -> 16 TMEM columns at 64 g + (c0 - 64 g) / 2
+        const uint32_t pc = static_cast<uint32_t>(cb + (c0 - cb) / 2);
+        if (KV) tmem_st16(lane_base + C::S_COL + pc, pk);
+        tmem_st16(lane_base + C::DP_COL + pc, dk);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8 * C::B_PDS_FULL);

@@ -121,15 +121,15 @@ struct FwdParams {
 };
 
 // Bounded wait on an mbarrier phase.  Gives up when the CTA-wide abort flag
-// is raised or after `limit_ns`; the first to give up records `code`.
+// is raised or after `limit_ns`; the first to give up records `code`.  Past
+// the first try (the fast path) the time and the flag are checked after every
+// try, so the bound holds to within one hardware suspension of the thread.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            unsigned long long limit_ns, unsigned code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
