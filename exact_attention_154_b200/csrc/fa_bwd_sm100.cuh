@@ -25,10 +25,10 @@
 // Keeping the 16-bit tiles in TMEM leaves shared memory for two slots of the
 // streamed pair in both kernels, so the next block loads during this one.
 //
-// Roles per CTA (320 threads): warps 0-7 compute P and dS (thread = TMEM
-// lane = tile row; warps 0-3 take columns 0-63 of each block, warps 4-7
-// columns 64-127), warp 8 streams tiles with TMA, warp 9 owns TMEM and one of
-// its threads issues every tcgen05.mma.  The streamed pair has two slots
+// Roles per CTA (576 threads): warps 0-15 compute P and dS (thread = TMEM
+// lane = tile row; warpgroup g takes columns 32 g .. 32 g + 31 of each
+// block), warp 16 streams tiles with TMA, warp 17 owns TMEM and one of its
+// threads issues every tcgen05.mma.  The streamed pair has two slots
 // where shared memory allows.  All mbarrier waits are bounded (wait_phase).
 #pragma once
 
@@ -61,9 +61,12 @@ struct BwdCfg {
   static constexpr int CHUNKS = HD / 64;
   static constexpr int CHUNK_BYTES = 128 * 128;
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;   // one [128 x HD] 16-bit tile
-  // two compute warpgroups (key/query rows x 64 of the 128 columns each),
-  // then the producer warp and the MMA warp
-  static constexpr int COMPUTE_WARPS = 8;
+  // four compute warpgroups (key/query rows x 32 of the 128 columns each),
+  // then the producer warp and the MMA warp.  The element work of a block
+  // sits between its S / dP products and its accumulating products, so the
+  // more warps share it the shorter that gap.
+  static constexpr int COMPUTE_WARPS = 16;
+  static constexpr int GROUP_COLS = 128 / (COMPUTE_WARPS / 4);
   static constexpr int THREADS = 32 * (COMPUTE_WARPS + 2);
   static constexpr int PRODUCER_WARP = COMPUTE_WARPS, MMA_WARP = COMPUTE_WARPS + 1;
   // Shared memory: the resident pair (K, V for dK/dV; Q, dO for dQ), STAGES
@@ -71,7 +74,7 @@ struct BwdCfg {
   // (dK/dV), barriers.  Two streamed slots where they fit, so the next block
   // loads while this one is computed.
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int VEC_BYTES = KV ? COMPUTE_WARPS * 2 * 64 * 4 : 0;
+  static constexpr int VEC_BYTES = KV ? COMPUTE_WARPS * 2 * GROUP_COLS * 4 : 0;
   static constexpr int B_RES_FULL = 0, B_STR_FULL = 1 /* [stage] */, B_STR_EMPTY = 3 /* [stage] */,
                        B_SD_FULL = 5, B_PDS_FULL = 6, B_DONE = 8, B_DRAIN = 9,
                        NUM_BARS = 10;
@@ -89,15 +92,15 @@ struct BwdCfg {
   static constexpr int SMEM_BYTES = END_OFF + 1024;  // + slack to align the base to 1024
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // TMEM columns: S (or S^T), dP (or dP^T), then the accumulators.  The
-  // 16-bit P (P^T) and dS (dS^T) overwrite the first half of each 64-column
-  // group's S / dP columns: columns [64 g, 64 g + 32) hold the packed values of
-  // columns [64 g, 64 g + 64) of the tile, written by compute group g.
+  // 16-bit P (P^T) and dS (dS^T) overwrite the first half of each 32-column
+  // group's S / dP columns: columns [32 g, 32 g + 16) hold the packed values of
+  // columns [32 g, 32 g + 32) of the tile, written by compute group g.
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0_COL = 256, ACC1_COL = 256 + HD;
   // TMEM column of the packed 16-bit operand for MMA K-step kk (16 columns
   // of the tile, 8 packed TMEM columns)
   __host__ __device__ static constexpr uint32_t packed_col(int kk) {
-    return 64u * static_cast<uint32_t>(kk / 4) + 8u * static_cast<uint32_t>(kk % 4);
+    return 32u * static_cast<uint32_t>(kk / 2) + 8u * static_cast<uint32_t>(kk % 2);
   }
 };
 
@@ -129,17 +132,18 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, 
     tma_load_4d(dst + c * (128 * 128), map, bar, c * 64, row0, h, b);
 }
 
-// Writes 32 fp32 accumulator columns of one row (times `mul`) as 16-bit values.
-template <bool BF16>
-__device__ __forceinline__ void store_acc32(void* dst_row, const uint32_t* acc, float mul) {
-  uint4 w[4];
+// Writes NC (16 or 32) fp32 accumulator columns of one row (times `mul`) as
+// 16-bit values.
+template <bool BF16, int NC>
+__device__ __forceinline__ void store_acc(void* dst_row, const uint32_t* acc, float mul) {
+  uint4 w[NC / 8];
   uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
+  for (int i = 0; i < NC / 2; ++i)
     wp[i] = pack2<BF16>(__uint_as_float(acc[2 * i]) * mul, __uint_as_float(acc[2 * i + 1]) * mul);
   uint4* dst = reinterpret_cast<uint4*>(dst_row);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) dst[i] = w[i];
+  for (int i = 0; i < NC / 8; ++i) dst[i] = w[i];
 }
 
 // KV = true: the dK/dV kernel (CTA per key block, streams Q and dO).
@@ -154,10 +158,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   uint8_t* smem = smem_raw + (base - raw);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-  // this warp's copy of the statistics of its 64 columns (no cross-warp
+  // this warp's copy of the statistics of its columns (no cross-warp
   // barrier, so a warp that leaves on an abandoned wait cannot strand the others)
-  float* lse2_s = reinterpret_cast<float*>(smem + C::VEC_OFF) + (threadIdx.x / 32) * 128;
-  float* dsum_s = lse2_s + 64;
+  float* lse2_s = reinterpret_cast<float*>(smem + C::VEC_OFF) + (threadIdx.x / 32) * 2 * C::GROUP_COLS;
+  float* dsum_s = lse2_s + C::GROUP_COLS;
   const uint32_t bars = base + C::BAR_OFF;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const unsigned long long lim = p.wait_limit_ns;
@@ -296,8 +300,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       }
     }
   } else {
-    // compute warps: thread = tile row = TMEM lane; this warpgroup's 64 columns
-    const int quad = warp % 4, cb = 64 * (warp / 4);
+    // compute warps: thread = tile row = TMEM lane; this warpgroup's columns
+    constexpr int GC = C::GROUP_COLS;
+    static_assert(GC == 32, "one 32-column pass per block");
+    const int quad = warp % 4, grp = warp / 4, cb = GC * grp;
     const int r = quad * 32 + lane;
     const uint32_t lane_base = tmem + ((static_cast<uint32_t>(quad) * 32u) << 16);
     const float sl2 = p.scale_log2;
@@ -317,7 +323,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         // query rows past N)
         __syncwarp();
 #pragma unroll
-        for (int c = lane; c < 64; c += 32) {
+        for (int c = lane; c < GC; c += 32) {
           const int qi = other0 + cb + c;
           lse2_s[c] = qi < p.N ? p.lse[vec0 + qi] * kLog2e : INFINITY;
           dsum_s[c] = qi < p.N ? p.dsum[vec0 + qi] : 0.f;
@@ -330,20 +336,20 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       tc_fence_after_sync();
       // (the previous step's 16-bit tiles in TMEM were read by its products,
       // which the MMA thread issued before this step's S / dP)
-#pragma unroll 1
-      for (int c0 = cb; c0 < cb + 64; c0 += 32) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32_sync(lane_base + C::S_COL + c0, sv);
-        tmem_ld32_sync(lane_base + C::DP_COL + c0, dv);
+      {
+        // S and dP of this thread's row over the group's 32 columns, one wait
+        uint32_t sd[64];
+        tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + C::DP_COL + cb, sd);
+        tmem_ld64_wait(sd);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           float pp[2], ds[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int c = c0 + 2 * q + e;
-            const float s = __uint_as_float(sv[2 * q + e]);
-            const float dpv = __uint_as_float(dv[2 * q + e]);
+            const int c = cb + 2 * q + e;
+            const float s = __uint_as_float(sd[2 * q + e]);
+            const float dpv = __uint_as_float(sd[32 + 2 * q + e]);
             float pv;
             if (KV) {
               // row = key my_row, column = query other0 + c
@@ -362,11 +368,9 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           pk[q] = pack2<BF16>(pp[0], pp[1]);
           dk[q] = pack2<BF16>(ds[0], ds[1]);
         }
-        // packed over the columns of this group already read: 32 tile
-        // columns -> 16 TMEM columns at 64 g + (c0 - 64 g) / 2
-        const uint32_t pc = static_cast<uint32_t>(cb + (c0 - cb) / 2);
-        if (KV) tmem_st16(lane_base + C::S_COL + pc, pk);
-        tmem_st16(lane_base + C::DP_COL + pc, dk);
+        // packed over the first 16 of the group's columns, already read
+        if (KV) tmem_st16(lane_base + C::S_COL + cb, pk);
+        tmem_st16(lane_base + C::DP_COL + cb, dk);
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -379,17 +383,32 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         tc_fence_after_sync();
         using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
         const long long row_off = (vec0 + my_row) * HD;
-#pragma unroll 1
-        for (int c = (warp / 4) * (HD / 2); c < (warp / 4 + 1) * (HD / 2); c += 32) {
+        // this group's quarter of the accumulator columns
+        constexpr int EC = HD / (C::COMPUTE_WARPS / 4);
+        const int c = grp * EC;
+        if constexpr (EC == 32) {
           uint32_t a0[32], a1[32];
           tmem_ld32_sync(lane_base + C::ACC0_COL + c, a0);
           if (KV) tmem_ld32_sync(lane_base + C::ACC1_COL + c, a1);
           if (my_row < p.N) {
             if (KV) {
-              store_acc32<BF16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f);
-              store_acc32<BF16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale);
+              store_acc<BF16, 32>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f);
+              store_acc<BF16, 32>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale);
             } else {
-              store_acc32<BF16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale);
+              store_acc<BF16, 32>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale);
+            }
+          }
+        } else {
+          static_assert(EC == 16, "accumulator quarter");
+          uint32_t a0[16], a1[16];
+          tmem_ld16_sync(lane_base + C::ACC0_COL + c, a0);
+          if (KV) tmem_ld16_sync(lane_base + C::ACC1_COL + c, a1);
+          if (my_row < p.N) {
+            if (KV) {
+              store_acc<BF16, 16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f);
+              store_acc<BF16, 16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale);
+            } else {
+              store_acc<BF16, 16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale);
             }
           }
         }

@@ -236,6 +236,21 @@ __device__ __forceinline__ void tmem_ld64_nowait(uint32_t taddr, uint32_t (&r)[6
       : "r"(taddr), "r"(taddr + 32)
       : "memory");
 }
+// 32 consecutive columns from each of two addresses into r[0..31] and
+// r[32..63], without waiting; tmem_ld64_wait() must follow.
+__device__ __forceinline__ void tmem_ld32x2_nowait(uint32_t taddr_a, uint32_t taddr_b,
+                                                   uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];"
+      : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24), FA_R8(32), FA_R8(40), FA_R8(48), FA_R8(56)
+      : "r"(taddr_a), "r"(taddr_b)
+      : "memory");
+}
 #define FA_RW8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), \
                   "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
 // Completes the loads issued so far; the registers are passed through so no
