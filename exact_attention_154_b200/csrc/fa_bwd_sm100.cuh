@@ -17,9 +17,10 @@
 // bwd_dkdv_kernel: one CTA per 128-key block j.  For every query block i it
 // computes S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM (tcgen05, SS),
 // forms P^T and dS^T in 16 bits (one thread per key row) and writes them back
-// into TMEM over the S^T / dP^T columns it has read, and accumulates
+// into TMEM over the dP^T columns it has read, and accumulates
 // dV_j += P^T dO_i and dK_j += dS^T Q_i in TMEM with P^T and dS^T as TMEM
-// operands (tcgen05.mma with A in tensor memory).
+// operands (tcgen05.mma with A in tensor memory).  The S^T columns are free
+// once read, so S^T for query block i+1 runs during block i's element work.
 // bwd_dq_kernel: one CTA per 128-query block i; recomputes S and dP the same
 // way for every key block j and accumulates dQ_i += dS K_j in TMEM.
 // Keeping the 16-bit tiles in TMEM leaves shared memory for two slots of the
@@ -76,8 +77,11 @@ struct BwdCfg {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int VEC_BYTES = KV ? COMPUTE_WARPS * 2 * GROUP_COLS * 4 : 0;
   static constexpr int B_RES_FULL = 0, B_STR_FULL = 1 /* [stage] */, B_STR_EMPTY = 3 /* [stage] */,
-                       B_SD_FULL = 5, B_PDS_FULL = 6, B_DONE = 8, B_DRAIN = 9,
-                       NUM_BARS = 10;
+                       B_SD_FULL = 5,
+                       // per block, one arrival per compute warp: S (S^T) and dP (dP^T)
+                       // read out of TMEM; P^T written (dK/dV only); dS (dS^T) written
+                       B_S_READ = 6, B_P_FULL = 7, B_DS_FULL = 8,
+                       B_DONE = 9, B_DRAIN = 10, NUM_BARS = 11;
   static constexpr int FIXED_BYTES = 2 * TILE_BYTES + VEC_BYTES +
                                      NUM_BARS * 8 + 16 + 1024;
   static constexpr int STAGES = FIXED_BYTES + 2 * STAGE_BYTES <= 232448 ? 2 : 1;
@@ -92,16 +96,20 @@ struct BwdCfg {
   static constexpr int SMEM_BYTES = END_OFF + 1024;  // + slack to align the base to 1024
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // TMEM columns: S (or S^T), dP (or dP^T), then the accumulators.  The
-  // 16-bit P (P^T) and dS (dS^T) overwrite the first half of each 32-column
-  // group's S / dP columns: columns [32 g, 32 g + 16) hold the packed values of
-  // columns [32 g, 32 g + 32) of the tile, written by compute group g.
+  // 16-bit tiles go into the dP (dP^T) columns only, each compute group over
+  // the 32 columns it has read itself: columns [32 g, 32 g + 16) of the dP
+  // region hold P^T (dK/dV kernel), columns [32 g + 16, 32 g + 32) dS (dS^T),
+  // packed two per column, for tile columns [32 g, 32 g + 32).  The S region
+  // is free as soon as it has been read, so the next block's S product runs
+  // while this block's element work does.
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0_COL = 256, ACC1_COL = 256 + HD;
-  // TMEM column of the packed 16-bit operand for MMA K-step kk (16 columns
-  // of the tile, 8 packed TMEM columns)
-  __host__ __device__ static constexpr uint32_t packed_col(int kk) {
-    return 32u * static_cast<uint32_t>(kk / 2) + 8u * static_cast<uint32_t>(kk % 2);
+  // TMEM column of the packed 16-bit P^T / dS operand for MMA K-step kk (16
+  // columns of the tile, 8 packed TMEM columns)
+  __host__ __device__ static constexpr uint32_t p_col(int kk) {
+    return DP_COL + 32u * static_cast<uint32_t>(kk / 2) + 8u * static_cast<uint32_t>(kk % 2);
   }
+  __host__ __device__ static constexpr uint32_t ds_col(int kk) { return p_col(kk) + 16u; }
 };
 
 // D_i = dO_i . O_i in fp32, one warp per row.
@@ -179,7 +187,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   if (threadIdx.x == 0) {
     // P / dS written: one arrival per compute warp; the rest are single
     for (int i = 0; i < C::NUM_BARS; ++i)
-      mbar_init(bars + 8 * i, i == C::B_PDS_FULL ? C::COMPUTE_WARPS : 1);
+      mbar_init(bars + 8 * i,
+                (i == C::B_S_READ || i == C::B_P_FULL || i == C::B_DS_FULL) ? C::COMPUTE_WARPS : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -238,58 +247,80 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       bool ok = wait_phase(bars + 8 * C::B_RES_FULL, 0, abort_flag, lim,
                            (kRoleMma << 8) | kSiteQFull);
       tc_fence_after_sync();
-      // K-major [128 x HD] operands: resident A-side tiles and streamed B-side tiles
+      // K-major [128 x HD] operands: resident A-side tiles ...
       const uint32_t a0 = sw128_desc_lo(base + C::SA_OFF, 16), a1 = sw128_desc_lo(base + C::SB_OFF, 16);
+      // the streamed pair of step `it` as K-major B of S / dP ...
+      auto bk = [&](int it, int t) {
+        return sw128_desc_lo(base + C::SSTR_OFF + (it % C::STAGES) * C::STAGE_BYTES + t * C::TILE_BYTES, 16);
+      };
+      auto wait_str = [&](int it) -> bool {
+        const bool r = wait_phase(bars + 8 * (C::B_STR_FULL + it % C::STAGES),
+                                  (it / C::STAGES) & 1, abort_flag, lim,
+                                  (kRoleMma << 8) | kSiteKvFull);
+        tc_fence_after_sync();
+        return r;
+      };
+      // dkdv: S^T = K Q^T (a0, t = 0), dP^T = V dO^T (a1, t = 1);
+      // dq: S = Q K^T, dP = dO V^T
+      auto issue_sq = [&](uint32_t d_col, uint32_t a, uint32_t b) {
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          mma_ss(tmem + d_col, desc_from_lo(a + off), desc_from_lo(b + off), idesc_sq,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      if (count > 0 && (ok = wait_str(0))) {
+        issue_sq(C::S_COL, a0, bk(0, 0));
+        issue_sq(C::DP_COL, a1, bk(0, 1));
+        tc_commit(bars + 8 * C::B_SD_FULL);
+      }
+      // Per step: the next S once this step's S has been read out; the
+      // accumulating products once their 16-bit operand is written; the next
+      // dP after them (its columns hold that operand until they have read it:
+      // tcgen05.mma operations from one thread run in issue order).
       for (int it = 0; ok && it < count; ++it) {
         const int stage = it % C::STAGES;
         const uint32_t slot = base + C::SSTR_OFF + stage * C::STAGE_BYTES;
-        // the streamed pair as K-major B of S / dP ...
-        const uint32_t b0 = sw128_desc_lo(slot, 16), b1 = sw128_desc_lo(slot + C::TILE_BYTES, 16);
         // ... and as MN-major B [K = 128 rows x N = HD] of the accumulating
         // products (Q for dK, K for dQ; dO for dV)
         const uint32_t mq = sw128_desc_lo(slot, C::CHUNK_BYTES);
         const uint32_t md = sw128_desc_lo(slot + C::TILE_BYTES, C::CHUNK_BYTES);
-        if (!(ok = wait_phase(bars + 8 * (C::B_STR_FULL + stage), (it / C::STAGES) & 1, abort_flag,
-                              lim, (kRoleMma << 8) | kSiteKvFull)))
-          break;
-        tc_fence_after_sync();
-        // dkdv: S^T = K Q^T, dP^T = V dO^T;  dq: S = Q K^T, dP = dO V^T
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + C::S_COL, desc_from_lo(a0 + off), desc_from_lo(b0 + off), idesc_sq,
-                 kk > 0 ? 1u : 0u);
+        const bool more = it + 1 < count;
+        if (more) {
+          if (!(ok = wait_str(it + 1))) break;
+          if (!(ok = wait_phase(bars + 8 * C::B_S_READ, it & 1, abort_flag, lim,
+                                (kRoleMma << 8) | kSiteSFree)))
+            break;
+          tc_fence_after_sync();
+          issue_sq(C::S_COL, a0, bk(it + 1, 0));
         }
+        if (KV) {
+          // dV += P^T dO
+          if (!(ok = wait_phase(bars + 8 * C::B_P_FULL, it & 1, abort_flag, lim,
+                                (kRoleMma << 8) | kSitePFull)))
+            break;
+          tc_fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + C::DP_COL, desc_from_lo(a1 + off), desc_from_lo(b1 + off), idesc_sq,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + C::ACC0_COL, tmem + C::p_col(kk), desc_from_lo(md + ((kk * 16 * 128) >> 4)),
+                   idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(bars + 8 * C::B_SD_FULL);
-        if (!(ok = wait_phase(bars + 8 * C::B_PDS_FULL, it & 1, abort_flag, lim,
+        // dK += dS^T Q (dkdv) or dQ += dS K (dq)
+        if (!(ok = wait_phase(bars + 8 * C::B_DS_FULL, it & 1, abort_flag, lim,
                               (kRoleMma << 8) | kSitePFull)))
           break;
         tc_fence_after_sync();
-        // the 16-bit tiles (in TMEM) contract over their 128 columns in 8
-        // K-steps; the next S / dP products, issued after these by this same
-        // thread, overwrite their columns only once these have read them
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t kb = (kk * 16 * 128) >> 4;
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t pcol = C::packed_col(kk);
-          if (KV) {
-            // dV += P^T dO, dK += dS^T Q
-            mma_ts(tmem + C::ACC0_COL, tmem + C::S_COL + pcol, desc_from_lo(md + kb), idesc_acc, acc);
-            mma_ts(tmem + C::ACC1_COL, tmem + C::DP_COL + pcol, desc_from_lo(mq + kb), idesc_acc, acc);
-          } else {
-            // dQ += dS K
-            mma_ts(tmem + C::ACC0_COL, tmem + C::DP_COL + pcol, desc_from_lo(mq + kb), idesc_acc, acc);
-          }
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + (KV ? C::ACC1_COL : C::ACC0_COL), tmem + C::ds_col(kk),
+                 desc_from_lo(mq + ((kk * 16 * 128) >> 4)), idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         // frees the streamed slot
         tc_commit(bars + 8 * (C::B_STR_EMPTY + stage));
+        if (more) {
+          issue_sq(C::DP_COL, a1, bk(it + 1, 1));
+          tc_commit(bars + 8 * C::B_SD_FULL);
+        }
       }
       if (ok) {
         tc_commit(bars + 8 * C::B_DONE);
@@ -334,48 +365,69 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
                       (kRoleSoftmax << 8) | kSiteSFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
-      // (the previous step's 16-bit tiles in TMEM were read by its products,
-      // which the MMA thread issued before this step's S / dP)
-      {
-        // S and dP of this thread's row over the group's 32 columns, one wait
-        uint32_t sd[64];
-        tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + C::DP_COL + cb, sd);
-        tmem_ld64_wait(sd);
-        uint32_t pk[16], dk[16];
+      // (the previous step's 16-bit tiles in the dP columns were read by its
+      // products, which the MMA thread issued before this step's dP)
+      // S and dP of this thread's row over the group's 32 columns, one wait
+      uint32_t sd[64];
+      tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + C::DP_COL + cb, sd);
+      tmem_ld64_wait(sd);
+      // both are in registers: the next S may overwrite the S columns
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * C::B_S_READ);
+      // P (kept in fp32 over the S registers for dS)
+      uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          float pp[2], ds[2];
+      for (int q = 0; q < 16; ++q) {
+        float pp[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = cb + 2 * q + e;
-            const float s = __uint_as_float(sd[2 * q + e]);
-            const float dpv = __uint_as_float(sd[32 + 2 * q + e]);
-            float pv;
-            if (KV) {
-              // row = key my_row, column = query other0 + c
-              const bool vis = !p.causal || other0 + c >= my_row;
-              pv = vis ? ex2(s * sl2 - lse2_s[c - cb]) : 0.f;
-              ds[e] = pv * (dpv - dsum_s[c - cb]);
-            } else {
-              // row = query my_row, column = key other0 + c
-              const int key = other0 + c;
-              const bool vis = key < p.N && (!p.causal || key <= my_row);
-              pv = vis ? ex2(s * sl2 - my_lse2) : 0.f;
-              ds[e] = pv * (dpv - my_dsum);
-            }
-            pp[e] = pv;
+        for (int e = 0; e < 2; ++e) {
+          const int c = cb + 2 * q + e;
+          const float s = __uint_as_float(sd[2 * q + e]);
+          float pv;
+          if (KV) {
+            // row = key my_row, column = query other0 + c
+            const bool vis = !p.causal || other0 + c >= my_row;
+            pv = vis ? ex2(s * sl2 - lse2_s[c - cb]) : 0.f;
+          } else {
+            // row = query my_row, column = key other0 + c
+            const int key = other0 + c;
+            const bool vis = key < p.N && (!p.causal || key <= my_row);
+            pv = vis ? ex2(s * sl2 - my_lse2) : 0.f;
           }
-          pk[q] = pack2<BF16>(pp[0], pp[1]);
-          dk[q] = pack2<BF16>(ds[0], ds[1]);
+          pp[e] = pv;
+          sd[2 * q + e] = __float_as_uint(pv);
         }
-        // packed over the first 16 of the group's columns, already read
-        if (KV) tmem_st16(lane_base + C::S_COL + cb, pk);
-        tmem_st16(lane_base + C::DP_COL + cb, dk);
+        pk[q] = pack2<BF16>(pp[0], pp[1]);
       }
+      if (KV) {
+        // P^T over the first 16 of the group's dP^T columns (read above)
+        tmem_st16(lane_base + C::DP_COL + cb, pk);
+        tmem_st_wait();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * C::B_P_FULL);
+      }
+      // dS = P (dP - D)
+      uint32_t dk[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float ds[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = cb + 2 * q + e;
+          const float pv = __uint_as_float(sd[2 * q + e]);
+          const float dpv = __uint_as_float(sd[32 + 2 * q + e]);
+          ds[e] = pv * (dpv - (KV ? dsum_s[c - cb] : my_dsum));
+        }
+        dk[q] = pack2<BF16>(ds[0], ds[1]);
+      }
+      // over the last 16 of the group's dP columns
+      tmem_st16(lane_base + C::DP_COL + cb + 16, dk);
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * C::B_PDS_FULL);
+      if (lane == 0) mbar_arrive(bars + 8 * C::B_DS_FULL);
     }
     if (ok) {
       ok = wait_phase(bars + 8 * C::B_DONE, 0, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
