@@ -102,14 +102,23 @@ struct BwdCfg {
   // packed two per column, for tile columns [32 g, 32 g + 32).  The S region
   // is free as soon as it has been read, so the next block's S product runs
   // while this block's element work does.
+  // Where the accumulators leave 128 columns (the dQ kernel; the dK/dV kernel
+  // at d = 64) there are two dP regions, used by alternate blocks: the next
+  // block's dP is then issued with its S, before this block's accumulating
+  // products have read this block's packed tiles.
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0_COL = 256, ACC1_COL = 256 + HD;
-  // TMEM column of the packed 16-bit P^T / dS operand for MMA K-step kk (16
-  // columns of the tile, 8 packed TMEM columns)
-  __host__ __device__ static constexpr uint32_t p_col(int kk) {
-    return DP_COL + 32u * static_cast<uint32_t>(kk / 2) + 8u * static_cast<uint32_t>(kk % 2);
+  static constexpr int DP_BUFS = (KV ? 256 + 2 * HD : 256 + HD) + 128 <= 512 ? 2 : 1;
+  static constexpr uint32_t DP2_COL = KV ? 256 + 2 * HD : 256 + HD;
+  __host__ __device__ static constexpr uint32_t dp_col(int it) {
+    return (DP_BUFS == 2 && (it & 1)) ? DP2_COL : DP_COL;
   }
-  __host__ __device__ static constexpr uint32_t ds_col(int kk) { return p_col(kk) + 16u; }
+  // TMEM column of the packed 16-bit P^T / dS operand for MMA K-step kk (16
+  // columns of the tile, 8 packed TMEM columns) of step it
+  __host__ __device__ static constexpr uint32_t p_col(int it, int kk) {
+    return dp_col(it) + 32u * static_cast<uint32_t>(kk / 2) + 8u * static_cast<uint32_t>(kk % 2);
+  }
+  __host__ __device__ static constexpr uint32_t ds_col(int it, int kk) { return p_col(it, kk) + 16u; }
 };
 
 // D_i = dO_i . O_i in fp32, one warp per row.
@@ -272,12 +281,14 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       };
       if (count > 0 && (ok = wait_str(0))) {
         issue_sq(C::S_COL, a0, bk(0, 0));
-        issue_sq(C::DP_COL, a1, bk(0, 1));
+        issue_sq(C::dp_col(0), a1, bk(0, 1));
         tc_commit(bars + 8 * C::B_SD_FULL);
       }
-      // Per step: the next S once this step's S has been read out; the
-      // accumulating products once their 16-bit operand is written; the next
-      // dP after them (its columns hold that operand until they have read it:
+      // Per step: the next S once this step's S has been read out (and with
+      // two dP regions the next dP with it: its region's last packed tiles
+      // were read by products issued before); the accumulating products once
+      // their 16-bit operand is written; with one dP region the next dP after
+      // them (its columns hold that operand until they have read it:
       // tcgen05.mma operations from one thread run in issue order).
       for (int it = 0; ok && it < count; ++it) {
         const int stage = it % C::STAGES;
@@ -294,6 +305,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
             break;
           tc_fence_after_sync();
           issue_sq(C::S_COL, a0, bk(it + 1, 0));
+          if (C::DP_BUFS == 2) {
+            issue_sq(C::dp_col(it + 1), a1, bk(it + 1, 1));
+            tc_commit(bars + 8 * C::B_SD_FULL);
+          }
         }
         if (KV) {
           // dV += P^T dO
@@ -303,7 +318,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           tc_fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::ACC0_COL, tmem + C::p_col(kk), desc_from_lo(md + ((kk * 16 * 128) >> 4)),
+            mma_ts(tmem + C::ACC0_COL, tmem + C::p_col(it, kk), desc_from_lo(md + ((kk * 16 * 128) >> 4)),
                    idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         }
         // dK += dS^T Q (dkdv) or dQ += dS K (dq)
@@ -313,11 +328,11 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         tc_fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + (KV ? C::ACC1_COL : C::ACC0_COL), tmem + C::ds_col(kk),
+          mma_ts(tmem + (KV ? C::ACC1_COL : C::ACC0_COL), tmem + C::ds_col(it, kk),
                  desc_from_lo(mq + ((kk * 16 * 128) >> 4)), idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
         // frees the streamed slot
         tc_commit(bars + 8 * (C::B_STR_EMPTY + stage));
-        if (more) {
+        if (more && C::DP_BUFS == 1) {
           issue_sq(C::DP_COL, a1, bk(it + 1, 1));
           tc_commit(bars + 8 * C::B_SD_FULL);
         }
@@ -365,11 +380,12 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
                       (kRoleSoftmax << 8) | kSiteSFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
-      // (the previous step's 16-bit tiles in the dP columns were read by its
-      // products, which the MMA thread issued before this step's dP)
+      // (the 16-bit tiles last written to this step's dP columns were read by
+      // products that the MMA thread issued before this step's dP)
       // S and dP of this thread's row over the group's 32 columns, one wait
       uint32_t sd[64];
-      tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + C::DP_COL + cb, sd);
+      const uint32_t dpc = C::dp_col(it);
+      tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + dpc + cb, sd);
       tmem_ld64_wait(sd);
       // both are in registers: the next S may overwrite the S columns
       tc_fence_before_sync();
@@ -402,7 +418,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       }
       if (KV) {
         // P^T over the first 16 of the group's dP^T columns (read above)
-        tmem_st16(lane_base + C::DP_COL + cb, pk);
+        tmem_st16(lane_base + dpc + cb, pk);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
@@ -423,7 +439,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         dk[q] = pack2<BF16>(ds[0], ds[1]);
       }
       // over the last 16 of the group's dP columns
-      tmem_st16(lane_base + C::DP_COL + cb + 16, dk);
+      tmem_st16(lane_base + dpc + cb + 16, dk);
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
