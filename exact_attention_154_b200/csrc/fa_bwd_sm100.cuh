@@ -140,6 +140,15 @@ __global__ void __launch_bounds__(256) bwd_dsum_kernel(const void* __restrict__ 
   if (lane == 0) dsum[row] = acc;
 }
 
+// Of every 8 argument pairs of P, how many take the FMA-pipe exp2 (exp2_poly2)
+// instead of ex2.  Measured on B200 at d = 128 and 64: 1 of 8 no change, 2 and
+// 3 of 8 slower (the exponential unit does not bound these kernels), so none.
+#ifdef FA_BWD_POLY8
+constexpr int BWD_POLY8 = FA_BWD_POLY8;
+#else
+constexpr int BWD_POLY8 = 0;
+#endif
+
 // Loads one [128 x HD] tile of a 4-D tensor map into shared memory.
 template <int HD>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -391,28 +400,32 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars + 8 * C::B_S_READ);
-      // P (kept in fp32 over the S registers for dS)
+      // P (kept in fp32 over the S registers for dS); BWD_POLY8 of every 8
+      // argument pairs take the FMA-pipe exp2, the rest ex2
       uint32_t pk[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        float pp[2];
+        const float2 nl = KV ? make_float2(-lse2_s[2 * q], -lse2_s[2 * q + 1])
+                             : make_float2(-my_lse2, -my_lse2);
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sd[2 * q]), __uint_as_float(sd[2 * q + 1])),
+                                    make_float2(sl2, sl2), nl);
+        float2 ev;
+        if ((q % 8) >= 8 - BWD_POLY8) {
+          ev = exp2_poly2(x);
+        } else {
+          ev.x = ex2(x.x);
+          ev.y = ex2(x.y);
+        }
+        float pp[2] = {ev.x, ev.y};
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int c = cb + 2 * q + e;
-          const float s = __uint_as_float(sd[2 * q + e]);
-          float pv;
-          if (KV) {
-            // row = key my_row, column = query other0 + c
-            const bool vis = !p.causal || other0 + c >= my_row;
-            pv = vis ? ex2(s * sl2 - lse2_s[c - cb]) : 0.f;
-          } else {
-            // row = query my_row, column = key other0 + c
-            const int key = other0 + c;
-            const bool vis = key < p.N && (!p.causal || key <= my_row);
-            pv = vis ? ex2(s * sl2 - my_lse2) : 0.f;
-          }
-          pp[e] = pv;
-          sd[2 * q + e] = __float_as_uint(pv);
+          // dkdv: row = key my_row, column = query other0 + c (columns past N
+          // carry lse = +inf); dq: row = query my_row, column = key other0 + c
+          const bool vis = KV ? (!p.causal || other0 + c >= my_row)
+                              : (other0 + c < p.N && (!p.causal || other0 + c <= my_row));
+          pp[e] = vis ? pp[e] : 0.f;
+          sd[2 * q + e] = __float_as_uint(pp[e]);
         }
         pk[q] = pack2<BF16>(pp[0], pp[1]);
       }
