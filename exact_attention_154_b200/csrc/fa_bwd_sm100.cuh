@@ -23,14 +23,15 @@
 // once read, so S^T for query block i+1 runs during block i's element work.
 // bwd_dq_kernel: one CTA per 128-query block i; recomputes S and dP the same
 // way for every key block j and accumulates dQ_i += dS K_j in TMEM.
-// Keeping the 16-bit tiles in TMEM leaves shared memory for two slots of the
-// streamed pair in both kernels, so the next block loads during this one.
+// Keeping the 16-bit tiles in TMEM leaves shared memory for five streamed
+// tiles (three of Q / K, two of dO / V), so the blocks after this one load
+// while it is computed.
 //
 // Roles per CTA (576 threads): warps 0-15 compute P and dS (thread = TMEM
 // lane = tile row; warpgroup g takes columns 32 g .. 32 g + 31 of each
 // block), warp 16 streams tiles with TMA, warp 17 owns TMEM and one of its
-// threads issues every tcgen05.mma.  The streamed pair has two slots
-// where shared memory allows.  All mbarrier waits are bounded (wait_phase).
+// threads issues every tcgen05.mma.  All mbarrier waits are bounded
+// (wait_phase).
 #pragma once
 
 #include "fa_fwd_sm100.cuh"
@@ -68,32 +69,33 @@ struct BwdCfg {
   // more warps share it the shorter that gap.
   static constexpr int COMPUTE_WARPS = 16;
   static constexpr int GROUP_COLS = 128 / (COMPUTE_WARPS / 4);
+  static_assert(GROUP_COLS == 32, "a warp's columns: one per lane");
   static constexpr int THREADS = 32 * (COMPUTE_WARPS + 2);
   static constexpr int PRODUCER_WARP = COMPUTE_WARPS, MMA_WARP = COMPUTE_WARPS + 1;
-  // Shared memory: the resident pair (K, V for dK/dV; Q, dO for dQ), STAGES
-  // slots of the streamed pair (Q, dO / K, V), per-warp column statistics
-  // (dK/dV), barriers.  Two streamed slots where they fit, so the next block
-  // loads while this one is computed.
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int VEC_BYTES = KV ? COMPUTE_WARPS * 2 * GROUP_COLS * 4 : 0;
-  static constexpr int B_RES_FULL = 0, B_STR_FULL = 1 /* [stage] */, B_STR_EMPTY = 3 /* [stage] */,
-                       B_SD_FULL = 5,
+  // Shared memory: the resident pair (K, V for dK/dV; Q, dO for dQ), two
+  // rings of streamed tiles, barriers.  The A stream (Q for dK/dV, K for dQ)
+  // is the B operand of S and of the last accumulating product (dK / dQ), so
+  // a slot is held to the end of its step: three slots.  The B stream (dO /
+  // V) is the B operand of dP (and of dV), released earlier: two slots.  With
+  // two streamed steps in flight the next step's S can be issued during this
+  // step's element work without waiting for its load.
+  static constexpr int A_SLOTS = 3, B_SLOTS = 2;
+  static constexpr int B_RES_FULL = 0, B_A_FULL = 1 /* [A slot] */, B_A_EMPTY = 4,
+                       B_B_FULL = 7 /* [B slot] */, B_B_EMPTY = 9, B_SD_FULL = 11,
                        // per block, one arrival per compute warp: S (S^T) and dP (dP^T)
                        // read out of TMEM; P^T written (dK/dV only); dS (dS^T) written
-                       B_S_READ = 6, B_P_FULL = 7, B_DS_FULL = 8,
-                       B_DONE = 9, B_DRAIN = 10, NUM_BARS = 11;
-  static constexpr int FIXED_BYTES = 2 * TILE_BYTES + VEC_BYTES +
-                                     NUM_BARS * 8 + 16 + 1024;
-  static constexpr int STAGES = FIXED_BYTES + 2 * STAGE_BYTES <= 232448 ? 2 : 1;
-  static constexpr int SA_OFF = 0;                           // K (dkdv) / Q (dq)
-  static constexpr int SB_OFF = TILE_BYTES;                  // V (dkdv) / dO (dq)
-  static constexpr int SSTR_OFF = 2 * TILE_BYTES;            // slot s: Q / K at +s*STAGE_BYTES,
-                                                             // dO / V at +TILE_BYTES
-  static constexpr int VEC_OFF = SSTR_OFF + STAGES * STAGE_BYTES;
-  static constexpr int BAR_OFF = VEC_OFF + VEC_BYTES;
+                       B_S_READ = 12, B_P_FULL = 13, B_DS_FULL = 14,
+                       B_DONE = 15, B_DRAIN = 16, NUM_BARS = 17;
+  static constexpr int SA_OFF = 0;                            // K (dkdv) / Q (dq)
+  static constexpr int SB_OFF = TILE_BYTES;                   // V (dkdv) / dO (dq)
+  static constexpr int RA_OFF = 2 * TILE_BYTES;               // A ring: Q (dkdv) / K (dq)
+  static constexpr int RB_OFF = RA_OFF + A_SLOTS * TILE_BYTES;  // B ring: dO (dkdv) / V (dq)
+  static constexpr int BAR_OFF = RB_OFF + B_SLOTS * TILE_BYTES;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
   static constexpr int END_OFF = MISC_OFF + 16;
-  static constexpr int SMEM_BYTES = END_OFF + 1024;  // + slack to align the base to 1024
+  // slack to align the base to 1024: the dynamic shared memory base is 16-byte
+  // aligned, so at most 1008 bytes are skipped
+  static constexpr int SMEM_BYTES = END_OFF + 1008;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // TMEM columns: S (or S^T), dP (or dP^T), then the accumulators.  The
   // 16-bit tiles go into the dP (dP^T) columns only, each compute group over
@@ -184,10 +186,6 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   uint8_t* smem = smem_raw + (base - raw);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
-  // this warp's copy of the statistics of its columns (no cross-warp
-  // barrier, so a warp that leaves on an abandoned wait cannot strand the others)
-  float* lse2_s = reinterpret_cast<float*>(smem + C::VEC_OFF) + (threadIdx.x / 32) * 2 * C::GROUP_COLS;
-  float* dsum_s = lse2_s + C::GROUP_COLS;
   const uint32_t bars = base + C::BAR_OFF;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const unsigned long long lim = p.wait_limit_ns;
@@ -228,33 +226,43 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   if (warp == C::PRODUCER_WARP) {
     if (lane == 0) {
       bool ok = true;
-      int issued = 0;
       // resident pair: K_j, V_j (dkdv) or Q_i, dO_i (dq)
       mbar_arrive_expect_tx(bars + 8 * C::B_RES_FULL, 2 * C::TILE_BYTES);
       load_tile<HD>(base + C::SA_OFF, KV ? &p.tmap_k : &p.tmap_q, bars + 8 * C::B_RES_FULL,
                     blk * 128, h, b);
       load_tile<HD>(base + C::SB_OFF, KV ? &p.tmap_v : &p.tmap_do, bars + 8 * C::B_RES_FULL,
                     blk * 128, h, b);
-      for (int it = 0; it < count; ++it) {
-        const int stage = it % C::STAGES, use = it / C::STAGES;
-        if (use > 0 && !(ok = wait_phase(bars + 8 * (C::B_STR_EMPTY + stage), (use - 1) & 1,
-                                         abort_flag, lim, (kRoleProducer << 8) | kSiteKvEmpty)))
-          break;
+      // A_it then B_it, each into its ring once the slot's previous tile is
+      // released
+      int issued_a = 0, issued_b = 0;
+      for (int it = 0; ok && it < count; ++it) {
         const int row0 = (first + it) * 128;
-        const uint32_t full = bars + 8 * (C::B_STR_FULL + stage);
-        const uint32_t slot = base + C::SSTR_OFF + stage * C::STAGE_BYTES;
-        mbar_arrive_expect_tx(full, 2 * C::TILE_BYTES);
-        load_tile<HD>(slot, KV ? &p.tmap_q : &p.tmap_k, full, row0, h, b);
-        load_tile<HD>(slot + C::TILE_BYTES, KV ? &p.tmap_do : &p.tmap_v, full, row0, h, b);
-        ++issued;
+#pragma unroll 1
+        for (int ring = 0; ring < 2; ++ring) {
+          const int slots = ring ? C::B_SLOTS : C::A_SLOTS;
+          const int slot = it % slots, use = it / slots;
+          const int b_empty = ring ? C::B_B_EMPTY : C::B_A_EMPTY;
+          if (use > 0 && !(ok = wait_phase(bars + 8 * (b_empty + slot), (use - 1) & 1, abort_flag,
+                                           lim, (kRoleProducer << 8) | kSiteKvEmpty)))
+            break;
+          const uint32_t full = bars + 8 * ((ring ? C::B_B_FULL : C::B_A_FULL) + slot);
+          mbar_arrive_expect_tx(full, C::TILE_BYTES);
+          load_tile<HD>(base + (ring ? C::RB_OFF : C::RA_OFF) + slot * C::TILE_BYTES,
+                        ring ? (KV ? &p.tmap_do : &p.tmap_v) : (KV ? &p.tmap_q : &p.tmap_k), full,
+                        row0, h, b);
+          ++(ring ? issued_b : issued_a);
+        }
       }
       if (!ok) {
         // let the loads in flight land before the shared memory goes away
         volatile int no_abort = 0;
         wait_phase(bars + 8 * C::B_RES_FULL, 0, &no_abort, 10000000ull,
                    (kRoleProducer << 8) | kSiteDrain);
-        for (int k = issued > C::STAGES ? issued - C::STAGES : 0; k < issued; ++k)
-          wait_phase(bars + 8 * (C::B_STR_FULL + k % C::STAGES), (k / C::STAGES) & 1, &no_abort,
+        for (int k = issued_a > C::A_SLOTS ? issued_a - C::A_SLOTS : 0; k < issued_a; ++k)
+          wait_phase(bars + 8 * (C::B_A_FULL + k % C::A_SLOTS), (k / C::A_SLOTS) & 1, &no_abort,
+                     10000000ull, (kRoleProducer << 8) | kSiteDrain);
+        for (int k = issued_b > C::B_SLOTS ? issued_b - C::B_SLOTS : 0; k < issued_b; ++k)
+          wait_phase(bars + 8 * (C::B_B_FULL + k % C::B_SLOTS), (k / C::B_SLOTS) & 1, &no_abort,
                      10000000ull, (kRoleProducer << 8) | kSiteDrain);
       }
     }
@@ -267,31 +275,38 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       tc_fence_after_sync();
       // K-major [128 x HD] operands: resident A-side tiles ...
       const uint32_t a0 = sw128_desc_lo(base + C::SA_OFF, 16), a1 = sw128_desc_lo(base + C::SB_OFF, 16);
-      // the streamed pair of step `it` as K-major B of S / dP ...
-      auto bk = [&](int it, int t) {
-        return sw128_desc_lo(base + C::SSTR_OFF + (it % C::STAGES) * C::STAGE_BYTES + t * C::TILE_BYTES, 16);
-      };
-      auto wait_str = [&](int it) -> bool {
-        const bool r = wait_phase(bars + 8 * (C::B_STR_FULL + it % C::STAGES),
-                                  (it / C::STAGES) & 1, abort_flag, lim,
-                                  (kRoleMma << 8) | kSiteKvFull);
+      // the streamed tiles of step `it`: K-major B of S (A ring) / dP (B ring),
+      // MN-major B [K = 128 rows x N = HD] of the accumulating products (Q for
+      // dK, K for dQ from the A ring; dO for dV from the B ring)
+      auto ra = [&](int it) { return base + C::RA_OFF + (it % C::A_SLOTS) * C::TILE_BYTES; };
+      auto rb = [&](int it) { return base + C::RB_OFF + (it % C::B_SLOTS) * C::TILE_BYTES; };
+      auto wait_ring = [&](int it, int ring) -> bool {
+        const int slots = ring ? C::B_SLOTS : C::A_SLOTS;
+        const bool r = wait_phase(bars + 8 * ((ring ? C::B_B_FULL : C::B_A_FULL) + it % slots),
+                                  (it / slots) & 1, abort_flag, lim, (kRoleMma << 8) | kSiteKvFull);
         tc_fence_after_sync();
         return r;
       };
-      // dkdv: S^T = K Q^T (a0, t = 0), dP^T = V dO^T (a1, t = 1);
+      // dkdv: S^T = K Q^T (a0, A ring), dP^T = V dO^T (a1, B ring);
       // dq: S = Q K^T, dP = dO V^T
-      auto issue_sq = [&](uint32_t d_col, uint32_t a, uint32_t b) {
+      auto issue_sq = [&](uint32_t d_col, uint32_t a, uint32_t bt) {
+        const uint32_t bd = sw128_desc_lo(bt, 16);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = ((kk / 4) * C::CHUNK_BYTES + (kk % 4) * 32) >> 4;
-          mma_ss(tmem + d_col, desc_from_lo(a + off), desc_from_lo(b + off), idesc_sq,
+          mma_ss(tmem + d_col, desc_from_lo(a + off), desc_from_lo(bd + off), idesc_sq,
                  kk > 0 ? 1u : 0u);
         }
       };
-      if (count > 0 && (ok = wait_str(0))) {
-        issue_sq(C::S_COL, a0, bk(0, 0));
-        issue_sq(C::dp_col(0), a1, bk(0, 1));
+      // dP of step it; in the dQ kernel the B-ring tile (V) has no other use
+      auto issue_dp = [&](int it) {
+        issue_sq(C::dp_col(it), a1, rb(it));
         tc_commit(bars + 8 * C::B_SD_FULL);
+        if (!KV) tc_commit(bars + 8 * (C::B_B_EMPTY + it % C::B_SLOTS));
+      };
+      if (count > 0) {
+        if ((ok = wait_ring(0, 0))) issue_sq(C::S_COL, a0, ra(0));
+        if (ok && (ok = wait_ring(0, 1))) issue_dp(0);
       }
       // Per step: the next S once this step's S has been read out (and with
       // two dP regions the next dP with it: its region's last packed tiles
@@ -300,27 +315,23 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       // them (its columns hold that operand until they have read it:
       // tcgen05.mma operations from one thread run in issue order).
       for (int it = 0; ok && it < count; ++it) {
-        const int stage = it % C::STAGES;
-        const uint32_t slot = base + C::SSTR_OFF + stage * C::STAGE_BYTES;
-        // ... and as MN-major B [K = 128 rows x N = HD] of the accumulating
-        // products (Q for dK, K for dQ; dO for dV)
-        const uint32_t mq = sw128_desc_lo(slot, C::CHUNK_BYTES);
-        const uint32_t md = sw128_desc_lo(slot + C::TILE_BYTES, C::CHUNK_BYTES);
+        const uint32_t mq = sw128_desc_lo(ra(it), C::CHUNK_BYTES);
+        const uint32_t md = sw128_desc_lo(rb(it), C::CHUNK_BYTES);
         const bool more = it + 1 < count;
         if (more) {
-          if (!(ok = wait_str(it + 1))) break;
+          if (!(ok = wait_ring(it + 1, 0))) break;
           if (!(ok = wait_phase(bars + 8 * C::B_S_READ, it & 1, abort_flag, lim,
                                 (kRoleMma << 8) | kSiteSFree)))
             break;
           tc_fence_after_sync();
-          issue_sq(C::S_COL, a0, bk(it + 1, 0));
+          issue_sq(C::S_COL, a0, ra(it + 1));
           if (C::DP_BUFS == 2) {
-            issue_sq(C::dp_col(it + 1), a1, bk(it + 1, 1));
-            tc_commit(bars + 8 * C::B_SD_FULL);
+            if (!(ok = wait_ring(it + 1, 1))) break;
+            issue_dp(it + 1);
           }
         }
         if (KV) {
-          // dV += P^T dO
+          // dV += P^T dO; then dO's slot is free
           if (!(ok = wait_phase(bars + 8 * C::B_P_FULL, it & 1, abort_flag, lim,
                                 (kRoleMma << 8) | kSitePFull)))
             break;
@@ -329,8 +340,9 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + C::ACC0_COL, tmem + C::p_col(it, kk), desc_from_lo(md + ((kk * 16 * 128) >> 4)),
                    idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bars + 8 * (C::B_B_EMPTY + it % C::B_SLOTS));
         }
-        // dK += dS^T Q (dkdv) or dQ += dS K (dq)
+        // dK += dS^T Q (dkdv) or dQ += dS K (dq); then the A slot is free
         if (!(ok = wait_phase(bars + 8 * C::B_DS_FULL, it & 1, abort_flag, lim,
                               (kRoleMma << 8) | kSitePFull)))
           break;
@@ -339,11 +351,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + (KV ? C::ACC1_COL : C::ACC0_COL), tmem + C::ds_col(it, kk),
                  desc_from_lo(mq + ((kk * 16 * 128) >> 4)), idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-        // frees the streamed slot
-        tc_commit(bars + 8 * (C::B_STR_EMPTY + stage));
+        tc_commit(bars + 8 * (C::B_A_EMPTY + it % C::A_SLOTS));
         if (more && C::DP_BUFS == 1) {
-          issue_sq(C::DP_COL, a1, bk(it + 1, 1));
-          tc_commit(bars + 8 * C::B_SD_FULL);
+          if (!(ok = wait_ring(it + 1, 1))) break;
+          issue_dp(it + 1);
         }
       }
       if (ok) {
@@ -373,17 +384,16 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
     bool ok = true;
     for (int it = 0; it < count; ++it) {
       const int other0 = (first + it) * 128;  // first streamed row of this step
+      // dkdv: the statistics of the streamed query block's columns, lane l
+      // holding column cb + l (+inf lse masks query rows past N); read by
+      // shuffles below
+      float col_lse2 = INFINITY, col_dsum = 0.f;
       if (KV) {
-        // per-column statistics of the streamed query block (+inf lse masks
-        // query rows past N)
-        __syncwarp();
-#pragma unroll
-        for (int c = lane; c < GC; c += 32) {
-          const int qi = other0 + cb + c;
-          lse2_s[c] = qi < p.N ? p.lse[vec0 + qi] * kLog2e : INFINITY;
-          dsum_s[c] = qi < p.N ? p.dsum[vec0 + qi] : 0.f;
+        const int qi = other0 + cb + lane;
+        if (qi < p.N) {
+          col_lse2 = p.lse[vec0 + qi] * kLog2e;
+          col_dsum = p.dsum[vec0 + qi];
         }
-        __syncwarp();
       }
       ok = wait_phase(bars + 8 * C::B_SD_FULL, it & 1, abort_flag, lim,
                       (kRoleSoftmax << 8) | kSiteSFull);
@@ -405,7 +415,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       uint32_t pk[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const float2 nl = KV ? make_float2(-lse2_s[2 * q], -lse2_s[2 * q + 1])
+        const float2 nl = KV ? make_float2(-__shfl_sync(0xffffffffu, col_lse2, 2 * q),
+                                           -__shfl_sync(0xffffffffu, col_lse2, 2 * q + 1))
                              : make_float2(-my_lse2, -my_lse2);
         const float2 x = __ffma2_rn(make_float2(__uint_as_float(sd[2 * q]), __uint_as_float(sd[2 * q + 1])),
                                     make_float2(sl2, sl2), nl);
@@ -447,7 +458,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           const int c = cb + 2 * q + e;
           const float pv = __uint_as_float(sd[2 * q + e]);
           const float dpv = __uint_as_float(sd[32 + 2 * q + e]);
-          ds[e] = pv * (dpv - (KV ? dsum_s[c - cb] : my_dsum));
+          ds[e] = pv * (dpv - (KV ? __shfl_sync(0xffffffffu, col_dsum, c - cb) : my_dsum));
         }
         dk[q] = pack2<BF16>(ds[0], ds[1]);
       }
