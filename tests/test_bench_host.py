@@ -55,3 +55,16 @@ def test_peaks_fall_back_when_the_measured_file_is_missing(monkeypatch, tmp_path
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     peaks, src = bench.load_peaks()
     assert src == "fallback" and peaks == bench.FALLBACK_PEAKS
+
+
+def test_peak_follows_the_length_of_the_timed_region():
+    peaks = {"bf16_tflops": 1662.1, "bf16_tflops_sustained": 1414.8, "hbm_gbs": 6453.1}
+    p, note = bench.pick_peak(peaks, "measured", 0.1)
+    assert p == 1662.1 and "burst" in note
+    p, note = bench.pick_peak(peaks, "measured", 1.08)
+    assert p == 1414.8 and "sustained" in note
+    # e4m3: the bf16 figure times the nominal fp8 / bf16 ratio
+    p, note = bench.pick_peak(peaks, "measured", 0.1, 2.0)
+    assert p == 2 * 1662.1 and "x 2" in note
+    p, _ = bench.pick_peak(dict(bench.FALLBACK_PEAKS), "fallback", 2.0)
+    assert p == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
