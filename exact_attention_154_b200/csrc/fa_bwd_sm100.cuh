@@ -83,9 +83,14 @@ struct BwdCfg {
   static constexpr int B_RES_FULL = 0, B_A_FULL = 1 /* [A slot] */, B_A_EMPTY = 4,
                        B_B_FULL = 7 /* [B slot] */, B_B_EMPTY = 9, B_SD_FULL = 11,
                        // per block, one arrival per compute warp: S (S^T) and dP (dP^T)
-                       // read out of TMEM; P^T written (dK/dV only); dS (dS^T) written
-                       B_S_READ = 12, B_P_FULL = 13, B_DS_FULL = 14,
-                       B_DONE = 15, B_DRAIN = 16, NUM_BARS = 17;
+                       // read out of TMEM; P^T written (dK/dV only); dS (dS^T) written.
+                       // P_FULL and DS_FULL have one barrier per block parity: with two dP
+                       // regions the next block's S and dP are in while this block's
+                       // element work runs, so a warp can arrive for block it+1 before
+                       // another has arrived for block it (never for it+2: that needs
+                       // every warp to have read block it+1's S).
+                       B_S_READ = 12, B_P_FULL = 13 /* [2] */, B_DS_FULL = 15 /* [2] */,
+                       B_DONE = 17, B_DRAIN = 18, NUM_BARS = 19;
   static constexpr int SA_OFF = 0;                            // K (dkdv) / Q (dq)
   static constexpr int SB_OFF = TILE_BYTES;                   // V (dkdv) / dO (dq)
   static constexpr int RA_OFF = 2 * TILE_BYTES;               // A ring: Q (dkdv) / K (dq)
@@ -203,8 +208,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   if (threadIdx.x == 0) {
     // P / dS written: one arrival per compute warp; the rest are single
     for (int i = 0; i < C::NUM_BARS; ++i)
-      mbar_init(bars + 8 * i,
-                (i == C::B_S_READ || i == C::B_P_FULL || i == C::B_DS_FULL) ? C::COMPUTE_WARPS : 1);
+      mbar_init(bars + 8 * i, (i >= C::B_S_READ && i < C::B_DONE) ? C::COMPUTE_WARPS : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -332,7 +336,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         }
         if (KV) {
           // dV += P^T dO; then dO's slot is free
-          if (!(ok = wait_phase(bars + 8 * C::B_P_FULL, it & 1, abort_flag, lim,
+          if (!(ok = wait_phase(bars + 8 * (C::B_P_FULL + (it & 1)), (it >> 1) & 1, abort_flag, lim,
                                 (kRoleMma << 8) | kSitePFull)))
             break;
           tc_fence_after_sync();
@@ -343,7 +347,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           tc_commit(bars + 8 * (C::B_B_EMPTY + it % C::B_SLOTS));
         }
         // dK += dS^T Q (dkdv) or dQ += dS K (dq); then the A slot is free
-        if (!(ok = wait_phase(bars + 8 * C::B_DS_FULL, it & 1, abort_flag, lim,
+        if (!(ok = wait_phase(bars + 8 * (C::B_DS_FULL + (it & 1)), (it >> 1) & 1, abort_flag, lim,
                               (kRoleMma << 8) | kSitePFull)))
           break;
         tc_fence_after_sync();
@@ -446,7 +450,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * C::B_P_FULL);
+        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + (it & 1)));
       }
       // dS = P (dP - D)
       uint32_t dk[16];
@@ -467,7 +471,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * C::B_DS_FULL);
+      if (lane == 0) mbar_arrive(bars + 8 * (C::B_DS_FULL + (it & 1)));
     }
     if (ok) {
       ok = wait_phase(bars + 8 * C::B_DONE, 0, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
