@@ -42,10 +42,13 @@ METRIC_BWD = "attention bwd TFLOP/s (bf16, 1×B200), 10·N²·d per head (5·N²
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "fa_fwd_sm100_traffic.md")
-KERNEL_SOURCES = ["exact_attention_154_b200/csrc/fa_fwd_sm100.cuh",
-                  "exact_attention_154_b200/csrc/fa_bwd_sm100.cuh",
-                  "exact_attention_154_b200/csrc/sm100_ptx.cuh",
-                  "exact_attention_154_b200/csrc/fa_api.cu"]
+# The sources each direction's kernels are built from: the forward kernel from
+# its header, the PTX wrappers and the host file; the backward kernels from
+# those and their own header.
+KERNEL_SOURCES = {"fwd": ["exact_attention_154_b200/csrc/fa_fwd_sm100.cuh",
+                          "exact_attention_154_b200/csrc/sm100_ptx.cuh",
+                          "exact_attention_154_b200/csrc/fa_api.cu"]}
+KERNEL_SOURCES["bwd"] = KERNEL_SOURCES["fwd"] + ["exact_attention_154_b200/csrc/fa_bwd_sm100.cuh"]
 
 
 def workloads_by_key():
@@ -99,9 +102,9 @@ def pick_peak(peaks, peak_src, region_s, ratio=1.0):
     return peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * ratio, note
 
 
-def kernel_source_hash():
+def kernel_source_hash(direction="fwd"):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[direction]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -109,13 +112,15 @@ def kernel_source_hash():
 
 def profiled_traffic(workload_key):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source and this workload; else None."""
+    the current source of that direction's kernels ("bwd:" keys: the backward)
+    and this workload; else None."""
     try:
         text = open(PROFILE_TRAFFIC).read()
     except OSError:
         return None
-    src = re.search(r"source_sha256:\s*([0-9a-f]+)", text)
-    if not src or src.group(1) != kernel_source_hash():
+    direction = "bwd" if workload_key.startswith("bwd:") else "fwd"
+    src = re.search(rf"source_sha256_{direction}:\s*([0-9a-f]+)", text)
+    if not src or src.group(1) != kernel_source_hash(direction):
         return None
     m = re.search(rf"traffic_bytes_per_launch\[{re.escape(workload_key)}\]:\s*([0-9.eE+]+)", text)
     return float(m.group(1)) if m else None

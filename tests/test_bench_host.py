@@ -25,12 +25,23 @@ def test_algorithmic_bytes_of_the_bench_workload():
 
 def test_traffic_record_is_gated_by_the_source_hash(tmp_path, monkeypatch):
     rec = tmp_path / "traffic.md"
-    rec.write_text(f"source_sha256: {bench.kernel_source_hash()}\n"
-                   "traffic_bytes_per_launch[sweep-n4096]: 123\n")
+    rec.write_text(f"source_sha256_fwd: {bench.kernel_source_hash('fwd')}\n"
+                   f"source_sha256_bwd: {bench.kernel_source_hash('bwd')}\n"
+                   "traffic_bytes_per_launch[sweep-n4096]: 123\n"
+                   "traffic_bytes_per_launch[bwd:sweep-n4096]: 456\n")
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(rec))
     assert bench.profiled_traffic("sweep-n4096") == 123.0
+    assert bench.profiled_traffic("bwd:sweep-n4096") == 456.0
     assert bench.profiled_traffic("sweep-n8192") is None
-    rec.write_text("source_sha256: 0000000000000000\ntraffic_bytes_per_launch[sweep-n4096]: 123\n")
+    # the backward hash covers the backward header too, the forward one does not
+    assert bench.kernel_source_hash("fwd") != bench.kernel_source_hash("bwd")
+    rec.write_text(f"source_sha256_fwd: {bench.kernel_source_hash('fwd')}\n"
+                   "source_sha256_bwd: 0000000000000000\n"
+                   "traffic_bytes_per_launch[sweep-n4096]: 123\n"
+                   "traffic_bytes_per_launch[bwd:sweep-n4096]: 456\n")
+    assert bench.profiled_traffic("sweep-n4096") == 123.0
+    assert bench.profiled_traffic("bwd:sweep-n4096") is None
+    rec.write_text("source_sha256_fwd: 0000000000000000\ntraffic_bytes_per_launch[sweep-n4096]: 123\n")
     assert bench.profiled_traffic("sweep-n4096") is None
     monkeypatch.setattr(bench, "PROFILE_TRAFFIC", str(tmp_path / "missing.md"))
     assert bench.profiled_traffic("sweep-n4096") is None
