@@ -16,7 +16,7 @@ with w_j the oracle's softmax weights, v_j the dequantised values and the
 last term the bf16 output rounding.  The test allows 1.25x that plus 1e-5
 (fp32 sums, ex2.approx).  The LSE uses the unrounded sum: 1e-3 relative as
 the 16-bit path.  At the bench size (N = 4096) the P rounding errors average
-over thousands of keys, and the benchmark spec mean-abs bound (2e-3) is checked
+over thousands of keys, and the 16-bit path's mean-abs bound (2e-3) is checked
 as well.
 """
 import numpy as np
