@@ -361,7 +361,9 @@ int launch_bwd_kernel(const BwdParams& p, DeviceState& st, cudaStream_t stream) 
   const int slot = (HD == 64 ? 0 : 4) + (BF16 ? 2 : 0) + (KV ? 1 : 0);
   const int rc = ensure_smem_attr(st.bwd_attr_set[slot], kernel, C::SMEM_BYTES);
   if (rc != FA_OK) return rc;
-  kernel<<<p.B * p.H * p.nblk, C::THREADS, C::SMEM_BYTES, stream>>>(p);
+  // persistent: one CTA per SM at most, each taking units in turn
+  const int grid = p.units < st.sm_count ? p.units : st.sm_count;
+  kernel<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -545,6 +547,7 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const fl
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.nblk = (N + 127) / 128;
+  p.units = B * H * p.nblk;
   p.wait_limit_ns = g_wait_limit_ns.load();
   const bool bf16 = dtype == FA_BF16;
   if (d == 64) return bf16 ? launch_bwd<64, true>(p, *st, s) : launch_bwd<64, false>(p, *st, s);

@@ -54,6 +54,7 @@ struct BwdParams {
   float scale;
   float scale_log2;     // scale * log2(e)
   int nblk;             // 128-row blocks per (b, h)
+  int units;            // B * H * nblk: one unit = one resident key (dK/dV) or query (dQ) block
   unsigned long long wait_limit_ns;
 };
 
@@ -90,7 +91,9 @@ struct BwdCfg {
                        // another has arrived for block it (never for it+2: that needs
                        // every warp to have read block it+1's S).
                        B_S_READ = 12, B_P_FULL = 13 /* [2] */, B_DS_FULL = 15 /* [2] */,
-                       B_DONE = 17, B_DRAIN = 18, NUM_BARS = 19;
+                       B_DONE = 17, B_DRAIN = 18,
+                       // the resident pair's last readers (a unit's last S and dP) ended
+                       B_RES_EMPTY = 19, NUM_BARS = 20;
   static constexpr int SA_OFF = 0;                            // K (dkdv) / Q (dq)
   static constexpr int SB_OFF = TILE_BYTES;                   // V (dkdv) / dO (dq)
   static constexpr int RA_OFF = 2 * TILE_BYTES;               // A ring: Q (dkdv) / K (dq)
@@ -179,8 +182,50 @@ __device__ __forceinline__ void store_acc(void* dst_row, const uint32_t* acc, fl
   for (int i = 0; i < NC / 8; ++i) dst[i] = w[i];
 }
 
-// KV = true: the dK/dV kernel (CTA per key block, streams Q and dO).
-// KV = false: the dQ kernel (CTA per query block, streams K and V).
+// One unit of work: a resident key block (dK/dV) or query block (dQ) of one
+// (b, h), and the streamed blocks it meets.
+struct BwdUnit {
+  int bh, blk, b, h;
+  int first, count;  // streamed blocks first .. first + count - 1
+};
+
+// Units in the order they are handed out.  Non-causal: (b, h)-major, so the
+// units running at once share a head's streamed tiles in L2.  Causal: the
+// units with the most blocks first (key block 0 of every head for dK/dV, the
+// last query block for dQ), so that with the snake hand-out below the
+// persistent CTAs get equal work.
+__device__ __forceinline__ BwdUnit bwd_unit(const BwdParams& p, int u, bool kv) {
+  BwdUnit w;
+  if (p.causal) {
+    const int nbh = p.B * p.H;
+    const int rank = u / nbh;
+    w.bh = u - rank * nbh;
+    w.blk = kv ? rank : p.nblk - 1 - rank;
+  } else {
+    w.bh = u / p.nblk;
+    w.blk = u - w.bh * p.nblk;
+  }
+  w.b = w.bh / p.H;
+  w.h = w.bh - w.b * p.H;
+  // causal: key block j meets query blocks j .. nblk-1, query block i meets
+  // key blocks 0 .. i
+  w.first = (kv && p.causal) ? w.blk : 0;
+  const int last = (!kv && p.causal) ? w.blk : p.nblk - 1;
+  w.count = last - w.first + 1;
+  return w;
+}
+
+// Persistent hand-out: round r gives CTA c unit r * G + c, in reverse CTA
+// order on odd rounds.
+__device__ __forceinline__ int bwd_unit_of(int round, int cta, int G) {
+  return round * G + ((round & 1) ? (G - 1 - cta) : cta);
+}
+
+// KV = true: the dK/dV kernel (units: key blocks, streams Q and dO).
+// KV = false: the dQ kernel (units: query blocks, streams K and V).
+// Persistent: min(units, SMs) CTAs, each taking units in turn; every role
+// counts the streamed steps over all its units, so ring slots and per-step
+// barrier phases run on across units.
 template <int HD, bool BF16, bool KV>
 __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ BwdParams p) {
@@ -195,15 +240,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const unsigned long long lim = p.wait_limit_ns;
 
-  // this CTA's (b, h) and resident block; the streamed blocks it visits
-  const int bh = blockIdx.x / p.nblk;
-  const int blk = blockIdx.x - bh * p.nblk;
-  const int b = bh / p.H, h = bh - b * p.H;
-  // causal: key block j meets query blocks j .. nblk-1, query block i meets
-  // key blocks 0 .. i
-  const int first = (KV && p.causal) ? blk : 0;
-  const int last = (!KV && p.causal) ? blk : p.nblk - 1;
-  const int count = last - first + 1;
+  const int G = gridDim.x, cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
     // P / dS written: one arrival per compute warp; the rest are single
@@ -230,43 +267,56 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   if (warp == C::PRODUCER_WARP) {
     if (lane == 0) {
       bool ok = true;
-      // resident pair: K_j, V_j (dkdv) or Q_i, dO_i (dq)
-      mbar_arrive_expect_tx(bars + 8 * C::B_RES_FULL, 2 * C::TILE_BYTES);
-      load_tile<HD>(base + C::SA_OFF, KV ? &p.tmap_k : &p.tmap_q, bars + 8 * C::B_RES_FULL,
-                    blk * 128, h, b);
-      load_tile<HD>(base + C::SB_OFF, KV ? &p.tmap_v : &p.tmap_do, bars + 8 * C::B_RES_FULL,
-                    blk * 128, h, b);
-      // A_it then B_it, each into its ring once the slot's previous tile is
-      // released
-      int issued_a = 0, issued_b = 0;
-      for (int it = 0; ok && it < count; ++it) {
-        const int row0 = (first + it) * 128;
+      int g = 0, k = 0;                // streamed steps and units so far
+      int issued_a = 0, issued_b = 0;  // ring loads issued (= g after each unit)
+      for (int round = 0; ok && round * G < p.units; ++round) {
+        const int u = bwd_unit_of(round, cta, G);
+        if (u >= p.units) continue;
+        const BwdUnit w = bwd_unit(p, u, KV);
+        // resident pair: K_j, V_j (dkdv) or Q_i, dO_i (dq), once the previous
+        // unit's S and dP products have ended
+        if (k > 0 && !(ok = wait_phase(bars + 8 * C::B_RES_EMPTY, (k - 1) & 1, abort_flag, lim,
+                                       (kRoleProducer << 8) | kSiteQEmpty)))
+          break;
+        mbar_arrive_expect_tx(bars + 8 * C::B_RES_FULL, 2 * C::TILE_BYTES);
+        load_tile<HD>(base + C::SA_OFF, KV ? &p.tmap_k : &p.tmap_q, bars + 8 * C::B_RES_FULL,
+                      w.blk * 128, w.h, w.b);
+        load_tile<HD>(base + C::SB_OFF, KV ? &p.tmap_v : &p.tmap_do, bars + 8 * C::B_RES_FULL,
+                      w.blk * 128, w.h, w.b);
+        ++k;
+        // A_it then B_it, each into its ring once the slot's previous tile is
+        // released
+        for (int it = 0; ok && it < w.count; ++it) {
+          const int gs = g + it, row0 = (w.first + it) * 128;
 #pragma unroll 1
-        for (int ring = 0; ring < 2; ++ring) {
-          const int slots = ring ? C::B_SLOTS : C::A_SLOTS;
-          const int slot = it % slots, use = it / slots;
-          const int b_empty = ring ? C::B_B_EMPTY : C::B_A_EMPTY;
-          if (use > 0 && !(ok = wait_phase(bars + 8 * (b_empty + slot), (use - 1) & 1, abort_flag,
-                                           lim, (kRoleProducer << 8) | kSiteKvEmpty)))
-            break;
-          const uint32_t full = bars + 8 * ((ring ? C::B_B_FULL : C::B_A_FULL) + slot);
-          mbar_arrive_expect_tx(full, C::TILE_BYTES);
-          load_tile<HD>(base + (ring ? C::RB_OFF : C::RA_OFF) + slot * C::TILE_BYTES,
-                        ring ? (KV ? &p.tmap_do : &p.tmap_v) : (KV ? &p.tmap_q : &p.tmap_k), full,
-                        row0, h, b);
-          ++(ring ? issued_b : issued_a);
+          for (int ring = 0; ring < 2; ++ring) {
+            const int slots = ring ? C::B_SLOTS : C::A_SLOTS;
+            const int slot = gs % slots, use = gs / slots;
+            const int b_empty = ring ? C::B_B_EMPTY : C::B_A_EMPTY;
+            if (use > 0 && !(ok = wait_phase(bars + 8 * (b_empty + slot), (use - 1) & 1, abort_flag,
+                                             lim, (kRoleProducer << 8) | kSiteKvEmpty)))
+              break;
+            const uint32_t full = bars + 8 * ((ring ? C::B_B_FULL : C::B_A_FULL) + slot);
+            mbar_arrive_expect_tx(full, C::TILE_BYTES);
+            load_tile<HD>(base + (ring ? C::RB_OFF : C::RA_OFF) + slot * C::TILE_BYTES,
+                          ring ? (KV ? &p.tmap_do : &p.tmap_v) : (KV ? &p.tmap_q : &p.tmap_k),
+                          full, row0, w.h, w.b);
+            ++(ring ? issued_b : issued_a);
+          }
         }
+        g += w.count;
       }
       if (!ok) {
         // let the loads in flight land before the shared memory goes away
         volatile int no_abort = 0;
-        wait_phase(bars + 8 * C::B_RES_FULL, 0, &no_abort, 10000000ull,
-                   (kRoleProducer << 8) | kSiteDrain);
-        for (int k = issued_a > C::A_SLOTS ? issued_a - C::A_SLOTS : 0; k < issued_a; ++k)
-          wait_phase(bars + 8 * (C::B_A_FULL + k % C::A_SLOTS), (k / C::A_SLOTS) & 1, &no_abort,
+        if (k > 0)
+          wait_phase(bars + 8 * C::B_RES_FULL, (k - 1) & 1, &no_abort, 10000000ull,
+                     (kRoleProducer << 8) | kSiteDrain);
+        for (int i = issued_a > C::A_SLOTS ? issued_a - C::A_SLOTS : 0; i < issued_a; ++i)
+          wait_phase(bars + 8 * (C::B_A_FULL + i % C::A_SLOTS), (i / C::A_SLOTS) & 1, &no_abort,
                      10000000ull, (kRoleProducer << 8) | kSiteDrain);
-        for (int k = issued_b > C::B_SLOTS ? issued_b - C::B_SLOTS : 0; k < issued_b; ++k)
-          wait_phase(bars + 8 * (C::B_B_FULL + k % C::B_SLOTS), (k / C::B_SLOTS) & 1, &no_abort,
+        for (int i = issued_b > C::B_SLOTS ? issued_b - C::B_SLOTS : 0; i < issued_b; ++i)
+          wait_phase(bars + 8 * (C::B_B_FULL + i % C::B_SLOTS), (i / C::B_SLOTS) & 1, &no_abort,
                      10000000ull, (kRoleProducer << 8) | kSiteDrain);
       }
     }
@@ -274,20 +324,18 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc_sq = f16_idesc(BF16, 128, 128, false);  // S-shaped: N = 128 rows
       const uint32_t idesc_acc = f16_idesc(BF16, 128, HD, true);   // accumulators: N = HD
-      bool ok = wait_phase(bars + 8 * C::B_RES_FULL, 0, abort_flag, lim,
-                           (kRoleMma << 8) | kSiteQFull);
-      tc_fence_after_sync();
+      bool ok = true;
       // K-major [128 x HD] operands: resident A-side tiles ...
       const uint32_t a0 = sw128_desc_lo(base + C::SA_OFF, 16), a1 = sw128_desc_lo(base + C::SB_OFF, 16);
-      // the streamed tiles of step `it`: K-major B of S (A ring) / dP (B ring),
-      // MN-major B [K = 128 rows x N = HD] of the accumulating products (Q for
-      // dK, K for dQ from the A ring; dO for dV from the B ring)
-      auto ra = [&](int it) { return base + C::RA_OFF + (it % C::A_SLOTS) * C::TILE_BYTES; };
-      auto rb = [&](int it) { return base + C::RB_OFF + (it % C::B_SLOTS) * C::TILE_BYTES; };
-      auto wait_ring = [&](int it, int ring) -> bool {
+      // the streamed tiles of global step gs: K-major B of S (A ring) / dP (B
+      // ring), MN-major B [K = 128 rows x N = HD] of the accumulating products
+      // (Q for dK, K for dQ from the A ring; dO for dV from the B ring)
+      auto ra = [&](int gs) { return base + C::RA_OFF + (gs % C::A_SLOTS) * C::TILE_BYTES; };
+      auto rb = [&](int gs) { return base + C::RB_OFF + (gs % C::B_SLOTS) * C::TILE_BYTES; };
+      auto wait_ring = [&](int gs, int ring) -> bool {
         const int slots = ring ? C::B_SLOTS : C::A_SLOTS;
-        const bool r = wait_phase(bars + 8 * ((ring ? C::B_B_FULL : C::B_A_FULL) + it % slots),
-                                  (it / slots) & 1, abort_flag, lim, (kRoleMma << 8) | kSiteKvFull);
+        const bool r = wait_phase(bars + 8 * ((ring ? C::B_B_FULL : C::B_A_FULL) + gs % slots),
+                                  (gs / slots) & 1, abort_flag, lim, (kRoleMma << 8) | kSiteKvFull);
         tc_fence_after_sync();
         return r;
       };
@@ -302,68 +350,92 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
                  kk > 0 ? 1u : 0u);
         }
       };
-      // dP of step it; in the dQ kernel the B-ring tile (V) has no other use
-      auto issue_dp = [&](int it) {
-        issue_sq(C::dp_col(it), a1, rb(it));
+      // dP of step gs; in the dQ kernel the B-ring tile (V) has no other use
+      auto issue_dp = [&](int gs) {
+        issue_sq(C::dp_col(gs), a1, rb(gs));
         tc_commit(bars + 8 * C::B_SD_FULL);
-        if (!KV) tc_commit(bars + 8 * (C::B_B_EMPTY + it % C::B_SLOTS));
+        if (!KV) tc_commit(bars + 8 * (C::B_B_EMPTY + gs % C::B_SLOTS));
       };
-      if (count > 0) {
-        if ((ok = wait_ring(0, 0))) issue_sq(C::S_COL, a0, ra(0));
-        if (ok && (ok = wait_ring(0, 1))) issue_dp(0);
-      }
-      // Per step: the next S once this step's S has been read out (and with
-      // two dP regions the next dP with it: its region's last packed tiles
-      // were read by products issued before); the accumulating products once
-      // their 16-bit operand is written; with one dP region the next dP after
-      // them (its columns hold that operand until they have read it:
-      // tcgen05.mma operations from one thread run in issue order).
-      for (int it = 0; ok && it < count; ++it) {
-        const uint32_t mq = sw128_desc_lo(ra(it), C::CHUNK_BYTES);
-        const uint32_t md = sw128_desc_lo(rb(it), C::CHUNK_BYTES);
-        const bool more = it + 1 < count;
-        if (more) {
-          if (!(ok = wait_ring(it + 1, 0))) break;
-          if (!(ok = wait_phase(bars + 8 * C::B_S_READ, it & 1, abort_flag, lim,
-                                (kRoleMma << 8) | kSiteSFree)))
-            break;
-          tc_fence_after_sync();
-          issue_sq(C::S_COL, a0, ra(it + 1));
-          if (C::DP_BUFS == 2) {
-            if (!(ok = wait_ring(it + 1, 1))) break;
-            issue_dp(it + 1);
+      int g = 0, k = 0;  // streamed steps and units so far
+      for (int round = 0; ok && round * G < p.units; ++round) {
+        const int u = bwd_unit_of(round, cta, G);
+        if (u >= p.units) continue;
+        const int count = bwd_unit(p, u, KV).count;
+        // The unit's resident pair.  (The previous unit's last S was read out
+        // before its last dK / dQ, which waited for every warp's dS of that
+        // step; its accumulators are read out by each warp's epilogue before
+        // that warp's P / dS of this unit's first step, which this unit's
+        // first accumulating products wait for.)
+        if (!(ok = wait_phase(bars + 8 * C::B_RES_FULL, k & 1, abort_flag, lim,
+                              (kRoleMma << 8) | kSiteQFull)))
+          break;
+        tc_fence_after_sync();
+        ++k;
+        if (!(ok = wait_ring(g, 0))) break;
+        issue_sq(C::S_COL, a0, ra(g));
+        if (!(ok = wait_ring(g, 1))) break;
+        issue_dp(g);
+        // the resident pair is free once the unit's last S and dP have ended
+        if (count == 1) tc_commit(bars + 8 * C::B_RES_EMPTY);
+        // Per step: the next S once this step's S has been read out (and with
+        // two dP regions the next dP with it: its region's last packed tiles
+        // were read by products issued before); the accumulating products once
+        // their 16-bit operand is written; with one dP region the next dP after
+        // them (its columns hold that operand until they have read it:
+        // tcgen05.mma operations from one thread run in issue order).
+        for (int it = 0; ok && it < count; ++it) {
+          const int gs = g + it;
+          const uint32_t mq = sw128_desc_lo(ra(gs), C::CHUNK_BYTES);
+          const uint32_t md = sw128_desc_lo(rb(gs), C::CHUNK_BYTES);
+          const bool more = it + 1 < count;
+          if (more) {
+            if (!(ok = wait_ring(gs + 1, 0))) break;
+            if (!(ok = wait_phase(bars + 8 * C::B_S_READ, gs & 1, abort_flag, lim,
+                                  (kRoleMma << 8) | kSiteSFree)))
+              break;
+            tc_fence_after_sync();
+            issue_sq(C::S_COL, a0, ra(gs + 1));
+            if (C::DP_BUFS == 2) {
+              if (!(ok = wait_ring(gs + 1, 1))) break;
+              issue_dp(gs + 1);
+              if (it + 2 == count) tc_commit(bars + 8 * C::B_RES_EMPTY);
+            }
           }
-        }
-        if (KV) {
-          // dV += P^T dO; then dO's slot is free
-          if (!(ok = wait_phase(bars + 8 * (C::B_P_FULL + (it & 1)), (it >> 1) & 1, abort_flag, lim,
+          if (KV) {
+            // dV += P^T dO; then dO's slot is free
+            if (!(ok = wait_phase(bars + 8 * (C::B_P_FULL + (gs & 1)), (gs >> 1) & 1, abort_flag,
+                                  lim, (kRoleMma << 8) | kSitePFull)))
+              break;
+            tc_fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + C::ACC0_COL, tmem + C::p_col(gs, kk),
+                     desc_from_lo(md + ((kk * 16 * 128) >> 4)), idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(bars + 8 * (C::B_B_EMPTY + gs % C::B_SLOTS));
+          }
+          // dK += dS^T Q (dkdv) or dQ += dS K (dq); then the A slot is free
+          if (!(ok = wait_phase(bars + 8 * (C::B_DS_FULL + (gs & 1)), (gs >> 1) & 1, abort_flag, lim,
                                 (kRoleMma << 8) | kSitePFull)))
             break;
           tc_fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + C::ACC0_COL, tmem + C::p_col(it, kk), desc_from_lo(md + ((kk * 16 * 128) >> 4)),
-                   idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bars + 8 * (C::B_B_EMPTY + it % C::B_SLOTS));
+            mma_ts(tmem + (KV ? C::ACC1_COL : C::ACC0_COL), tmem + C::ds_col(gs, kk),
+                   desc_from_lo(mq + ((kk * 16 * 128) >> 4)), idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bars + 8 * (C::B_A_EMPTY + gs % C::A_SLOTS));
+          if (more && C::DP_BUFS == 1) {
+            if (!(ok = wait_ring(gs + 1, 1))) break;
+            issue_dp(gs + 1);
+            if (it + 2 == count) tc_commit(bars + 8 * C::B_RES_EMPTY);
+          }
         }
-        // dK += dS^T Q (dkdv) or dQ += dS K (dq); then the A slot is free
-        if (!(ok = wait_phase(bars + 8 * (C::B_DS_FULL + (it & 1)), (it >> 1) & 1, abort_flag, lim,
-                              (kRoleMma << 8) | kSitePFull)))
-          break;
-        tc_fence_after_sync();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + (KV ? C::ACC1_COL : C::ACC0_COL), tmem + C::ds_col(it, kk),
-                 desc_from_lo(mq + ((kk * 16 * 128) >> 4)), idesc_acc, (it > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bars + 8 * (C::B_A_EMPTY + it % C::A_SLOTS));
-        if (more && C::DP_BUFS == 1) {
-          if (!(ok = wait_ring(it + 1, 1))) break;
-          issue_dp(it + 1);
-        }
-      }
-      if (ok) {
+        if (!ok) break;
+        // the unit's accumulators are complete once these products end
         tc_commit(bars + 8 * C::B_DONE);
-      } else {
+        g += count;
+      }
+      if (!ok) {
+        // wait for every MMA this thread issued before TMEM is released
         volatile int no_abort = 0;
         tc_commit(bars + 8 * C::B_DRAIN);
         wait_phase(bars + 8 * C::B_DRAIN, 0, &no_abort, 10000000ull, (kRoleMma << 8) | kSiteDrain);
@@ -378,16 +450,22 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
     const uint32_t lane_base = tmem + ((static_cast<uint32_t>(quad) * 32u) << 16);
     const float sl2 = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
-    const long long vec0 = static_cast<long long>(bh) * p.N;
-    const int my_row = blk * 128 + r;  // key row (dkdv) or query row (dq)
+    bool ok = true;
+    int g = 0, k = 0;  // streamed steps and units so far
+    for (int round = 0; ok && round * G < p.units; ++round) {
+    const int u = bwd_unit_of(round, cta, G);
+    if (u >= p.units) continue;
+    const BwdUnit w = bwd_unit(p, u, KV);
+    const long long vec0 = static_cast<long long>(w.bh) * p.N;
+    const int my_row = w.blk * 128 + r;  // key row (dkdv) or query row (dq)
     float my_lse2 = INFINITY, my_dsum = 0.f;
     if (!KV && my_row < p.N) {
       my_lse2 = p.lse[vec0 + my_row] * kLog2e;
       my_dsum = p.dsum[vec0 + my_row];
     }
-    bool ok = true;
-    for (int it = 0; it < count; ++it) {
-      const int other0 = (first + it) * 128;  // first streamed row of this step
+    for (int it = 0; it < w.count; ++it) {
+      const int gs = g + it;
+      const int other0 = (w.first + it) * 128;  // first streamed row of this step
       // dkdv: the statistics of the streamed query block's columns, lane l
       // holding column cb + l (+inf lse masks query rows past N); read by
       // shuffles below
@@ -399,7 +477,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           col_dsum = p.dsum[vec0 + qi];
         }
       }
-      ok = wait_phase(bars + 8 * C::B_SD_FULL, it & 1, abort_flag, lim,
+      ok = wait_phase(bars + 8 * C::B_SD_FULL, gs & 1, abort_flag, lim,
                       (kRoleSoftmax << 8) | kSiteSFull);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after_sync();
@@ -407,7 +485,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       // products that the MMA thread issued before this step's dP)
       // S and dP of this thread's row over the group's 32 columns, one wait
       uint32_t sd[64];
-      const uint32_t dpc = C::dp_col(it);
+      const uint32_t dpc = C::dp_col(gs);
       tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + dpc + cb, sd);
       tmem_ld64_wait(sd);
       // both are in registers: the next S may overwrite the S columns
@@ -450,7 +528,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + (it & 1)));
+        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + (gs & 1)));
       }
       // dS = P (dP - D)
       uint32_t dk[16];
@@ -471,11 +549,12 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
       tmem_st_wait();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * (C::B_DS_FULL + (it & 1)));
+      if (lane == 0) mbar_arrive(bars + 8 * (C::B_DS_FULL + (gs & 1)));
     }
     if (ok) {
-      ok = wait_phase(bars + 8 * C::B_DONE, 0, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
-      if (__all_sync(0xffffffffu, ok)) {
+      ok = wait_phase(bars + 8 * C::B_DONE, k & 1, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
         tc_fence_after_sync();
         using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
         const long long row_off = (vec0 + my_row) * HD;
@@ -509,6 +588,9 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           }
         }
       }
+    }
+    g += w.count;
+    ++k;
     }
   }
 

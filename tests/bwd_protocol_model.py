@@ -27,17 +27,21 @@ A_SLOTS, B_SLOTS = 3, 2
 
 class BwdSim:
     def __init__(s, count, kv, dp_bufs, seed, warps=4, skip_sread=False, early_a_empty=False,
-                 shared_full=False):
+                 shared_full=False, skip_res_empty=False):
         # skip_sread / early_a_empty / shared_full: deliberately broken
         # protocols (the next S issued without waiting for this step's S to be
         # read; the A slot released before dK / dQ read it; one P_FULL and one
         # DS_FULL barrier for all steps instead of one per step parity), for
         # the model's own negative tests
-        s.count, s.kv, s.dp_bufs, s.warps = count, kv, dp_bufs, warps
+        # count: blocks of the one unit, or a list of the units' block counts
+        # (a persistent CTA takes several units in turn)
+        s.units = list(count) if isinstance(count, (list, tuple)) else [count]
+        s.kv, s.dp_bufs, s.warps = kv, dp_bufs, warps
+        s.skip_res_empty = skip_res_empty
         s.skip_sread, s.early_a_empty, s.shared_full = skip_sread, early_a_empty, shared_full
         s.rng = random.Random(seed)
         s.b = {}
-        for n in ['RES', 'SD', 'DONE']: s.b[n] = Bar(n, 1)
+        for n in ['RES', 'RESE', 'SD', 'DONE']: s.b[n] = Bar(n, 1)
         # P / dS written: one barrier per step parity (a warp can run one step
         # ahead of another once the next step's S and dP are in)
         for n in ['SREAD', 'PFULL0', 'PFULL1', 'DSFULL0', 'DSFULL1']: s.b[n] = Bar(n, warps)
@@ -113,89 +117,122 @@ class BwdSim:
 
     # -------------------------------------------------------------- roles
     def producer(s):
-        s.b['RES'].expect(1); s.later(s.rng.randint(1, 40), lambda: s.b['RES'].tx_done(1))
-        for it in range(s.count):
-            for ring, slots in (('A', A_SLOTS), ('B', B_SLOTS)):
-                slot, use = it % slots, it // slots
-                if use > 0:
-                    e = f'{ring}E{slot}'
-                    s.phase_check(e, use - 1, 'prod')
-                    yield from s.wait(e, (use - 1) & 1, 'prod')
-                s.tma((ring, slot), f'{ring}F{slot}', it)
+        g = 0
+        for k, count in enumerate(s.units):
+            # the resident pair of unit k, once unit k-1's S and dP products
+            # (its only readers) have ended
+            if k > 0 and not s.skip_res_empty:
+                s.phase_check('RESE', k - 1, 'prod')
+                yield from s.wait('RESE', (k - 1) & 1, 'prod')
+            s.b['RES'].expect(1)
+
+            def land(k=k):
+                s.mem['RA'] = k; s.mem['RB'] = k
+                s.b['RES'].tx_done(1)
+            s.later(s.rng.randint(1, 40), land)
+            for it in range(count):
+                gs = g + it
+                for ring, slots in (('A', A_SLOTS), ('B', B_SLOTS)):
+                    slot, use = gs % slots, gs // slots
+                    if use > 0:
+                        e = f'{ring}E{slot}'
+                        s.phase_check(e, use - 1, 'prod')
+                        yield from s.wait(e, (use - 1) & 1, 'prod')
+                    s.tma((ring, slot), f'{ring}F{slot}', gs)
+            g += count
         yield ('done',)
 
     def mma_thread(s):
         kv = s.kv
-        yield from s.wait('RES', 0, 'mma')
 
-        def wait_ring(it, ring):
+        def wait_ring(gs, ring):
             slots = A_SLOTS if ring == 'A' else B_SLOTS
-            s.phase_check(f'{ring}F{it % slots}', it // slots, 'mma')
-            yield from s.wait(f'{ring}F{it % slots}', (it // slots) & 1, 'mma')
+            s.phase_check(f'{ring}F{gs % slots}', gs // slots, 'mma')
+            yield from s.wait(f'{ring}F{gs % slots}', (gs // slots) & 1, 'mma')
 
-        def issue_s(it):
-            s.mma(f'S({it})', [(('A', it % A_SLOTS), it)], [('S', ('S', it))])
+        def issue_s(gs, k):
+            s.mma(f'S({gs})', [(('A', gs % A_SLOTS), gs), ('RA', k)], [('S', ('S', gs))])
 
-        def issue_dp(it):
-            s.mma(f'dP({it})', [(('B', it % B_SLOTS), it)], [(s.dp(it), ('dP', it))])
+        def issue_dp(gs, k):
+            s.mma(f'dP({gs})', [(('B', gs % B_SLOTS), gs), ('RB', k)], [(s.dp(gs), ('dP', gs))])
             s.commit('SD')
-            if not kv: s.commit(f'BE{it % B_SLOTS}')
+            if not kv: s.commit(f'BE{gs % B_SLOTS}')
 
-        if s.count > 0:
-            yield from wait_ring(0, 'A'); issue_s(0)
-            yield from wait_ring(0, 'B'); issue_dp(0)
-        for it in range(s.count):
-            more = it + 1 < s.count
-            if more:
-                yield from wait_ring(it + 1, 'A')
-                if not s.skip_sread:
-                    s.phase_check('SREAD', it, 'mma')
-                    yield from s.wait('SREAD', it & 1, 'mma')
-                issue_s(it + 1)
-                if s.dp_bufs == 2:
-                    yield from wait_ring(it + 1, 'B'); issue_dp(it + 1)
-            if kv:
-                bar, ph = s.full('PFULL', it)
+        g = 0
+        for k, count in enumerate(s.units):
+            s.phase_check('RES', k, 'mma')
+            yield from s.wait('RES', k & 1, 'mma')
+            # (the previous unit's last S was read out before its last dK / dQ,
+            # which waited for every warp's dS of that step)
+            yield from wait_ring(g, 'A'); issue_s(g, k)
+            yield from wait_ring(g, 'B'); issue_dp(g, k)
+            if count == 1: s.commit('RESE')
+            for it in range(count):
+                gs = g + it
+                more = it + 1 < count
+                if more:
+                    yield from wait_ring(gs + 1, 'A')
+                    if not s.skip_sread:
+                        s.phase_check('SREAD', gs, 'mma')
+                        yield from s.wait('SREAD', gs & 1, 'mma')
+                    issue_s(gs + 1, k)
+                    if s.dp_bufs == 2:
+                        yield from wait_ring(gs + 1, 'B'); issue_dp(gs + 1, k)
+                        if it + 2 == count: s.commit('RESE')
+                if kv:
+                    bar, ph = s.full('PFULL', gs)
+                    s.phase_check(bar, ph, 'mma')
+                    yield from s.wait(bar, ph & 1, 'mma')
+                    s.mma(f'dV({gs})', [(('B', gs % B_SLOTS), gs)] +
+                          [((s.dp(gs), 'P', w), gs) for w in range(s.warps)], [('ACC', ('ACC', k))])
+                    s.commit(f'BE{gs % B_SLOTS}')
+                if s.early_a_empty: s.commit(f'AE{gs % A_SLOTS}')
+                bar, ph = s.full('DSFULL', gs)
                 s.phase_check(bar, ph, 'mma')
                 yield from s.wait(bar, ph & 1, 'mma')
-                s.mma(f'dV({it})', [(('B', it % B_SLOTS), it)] +
-                      [((s.dp(it), 'P', w), it) for w in range(s.warps)], [])
-                s.commit(f'BE{it % B_SLOTS}')
-            if s.early_a_empty: s.commit(f'AE{it % A_SLOTS}')
-            bar, ph = s.full('DSFULL', it)
-            s.phase_check(bar, ph, 'mma')
-            yield from s.wait(bar, ph & 1, 'mma')
-            s.mma(f'dK({it})', [(('A', it % A_SLOTS), it)] +
-                  [((s.dp(it), 'dS', w), it) for w in range(s.warps)], [])
-            if not s.early_a_empty: s.commit(f'AE{it % A_SLOTS}')
-            if more and s.dp_bufs == 1:
-                yield from wait_ring(it + 1, 'B'); issue_dp(it + 1)
-            yield ('work',)
-        s.commit('DONE')
+                s.mma(f'dK({gs})', [(('A', gs % A_SLOTS), gs)] +
+                      [((s.dp(gs), 'dS', w), gs) for w in range(s.warps)], [('ACC', ('ACC', k))])
+                if not s.early_a_empty: s.commit(f'AE{gs % A_SLOTS}')
+                if more and s.dp_bufs == 1:
+                    yield from wait_ring(gs + 1, 'B'); issue_dp(gs + 1, k)
+                    if it + 2 == count: s.commit('RESE')
+                yield ('work',)
+            s.commit('DONE')
+            g += count
         yield ('done',)
 
     def compute(s, w):
-        for it in range(s.count):
-            s.phase_check('SD', it, f'c{w}')
-            yield from s.wait('SD', it & 1, f'c{w}')
-            # the warps reach their loads at different times
-            for _ in range(s.rng.randint(0, 20)): yield ('work',)
-            # loads of S and of this step's dP region
-            s.expect('S', ('S', it), f'c{w} load S')
-            r = s.dp(it)
-            s.expect(r, ('dP', it), f'c{w} load dP')
-            yield ('work',)
-            s.b['SREAD'].arrive()
-            for _ in range(s.rng.randint(0, 20)): yield ('work',)
-            # packed tiles over this warp's own dP columns: a write of the
-            # region by an MMA would clobber them, so track them per warp
-            if s.kv:
-                s.mem[(r, 'P', w)] = it
-                s.b[s.full('PFULL', it)[0]].arrive()
+        g = 0
+        for k, count in enumerate(s.units):
+            for it in range(count):
+                gs = g + it
+                s.phase_check('SD', gs, f'c{w}')
+                yield from s.wait('SD', gs & 1, f'c{w}')
+                # the warps reach their loads at different times
+                for _ in range(s.rng.randint(0, 20)): yield ('work',)
+                # loads of S and of this step's dP region
+                s.expect('S', ('S', gs), f'c{w} load S')
+                r = s.dp(gs)
+                s.expect(r, ('dP', gs), f'c{w} load dP')
                 yield ('work',)
-            s.mem[(r, 'dS', w)] = it
-            s.b[s.full('DSFULL', it)[0]].arrive()
-        yield from s.wait('DONE', 0, f'c{w}')
+                s.b['SREAD'].arrive()
+                for _ in range(s.rng.randint(0, 20)): yield ('work',)
+                # packed tiles over this warp's own dP columns: a write of the
+                # region by an MMA would clobber them, so track them per warp
+                if s.kv:
+                    s.mem[(r, 'P', w)] = gs
+                    s.b[s.full('PFULL', gs)[0]].arrive()
+                    yield ('work',)
+                s.mem[(r, 'dS', w)] = gs
+                s.b[s.full('DSFULL', gs)[0]].arrive()
+            s.phase_check('DONE', k, f'c{w}')
+            yield from s.wait('DONE', k & 1, f'c{w}')
+            # epilogue: read the accumulators.  The next unit's first
+            # accumulating product waits for this warp's P / dS of that unit,
+            # written after this read, so no other hand-back is needed.
+            for _ in range(s.rng.randint(0, 20)): yield ('work',)
+            s.expect('ACC', ('ACC', k), f'c{w} epilogue')
+            g += count
         yield ('done',)
 
     def run(s, max_steps=400000):

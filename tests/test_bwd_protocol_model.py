@@ -40,3 +40,34 @@ def test_model_catches_a_broken_protocol(flaw, dp_bufs):
         r = sim.run()
         bad += (r != "ok") or bool(sim.errors)
     assert bad > 0
+
+
+UNITS = [[3, 1, 5, 2], [32, 32], [1, 1, 1, 1], [8, 7, 6, 5, 4, 3, 2, 1]]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda c: f"kv{int(c['kv'])}-dp{c['dp_bufs']}")
+@pytest.mark.parametrize("units", UNITS, ids=lambda u: "-".join(map(str, u)))
+def test_persistent_units_run_clean(shape, units):
+    """A persistent CTA takes several (key or query block) units in turn: the
+    next unit's resident tiles load once the last S / dP of this one have
+    ended; its first S follows this unit's last dK / dQ, which waited for
+    every warp to finish the last step; its first accumulating product
+    follows every warp's epilogue read of the accumulators through that
+    warp's P / dS arrivals for the new unit."""
+    for seed in range(4):
+        sim = bm.BwdSim(units, seed=seed, **shape)
+        r = sim.run()
+        assert r == "ok", (seed, r)
+        assert not sim.errors, (seed, sim.errors[:3])
+
+
+def test_model_catches_resident_tiles_reloaded_too_early():
+    """Negative control: loading the next unit's resident tiles without
+    waiting for the last S / dP products of this one to end shows an S or dP
+    reading the wrong unit's tile in some schedule."""
+    bad = 0
+    for seed in range(20):
+        sim = bm.BwdSim([4, 4, 4], kv=True, dp_bufs=1, seed=seed, skip_res_empty=True)
+        r = sim.run()
+        bad += (r != "ok") or bool(sim.errors)
+    assert bad > 0
