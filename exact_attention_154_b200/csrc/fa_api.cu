@@ -540,6 +540,9 @@ int run_bwd(const void* q, const void* k, const void* v, const void* o, const fl
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
+  // rows are HD 16-bit values (128 or 256 bytes), so the bases decide
+  p.out_vec32 = ((reinterpret_cast<uintptr_t>(dq) | reinterpret_cast<uintptr_t>(dk) |
+                  reinterpret_cast<uintptr_t>(dv)) & 31u) == 0;
   p.B = B;
   p.H = H;
   p.N = N;

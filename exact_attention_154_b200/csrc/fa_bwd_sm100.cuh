@@ -55,6 +55,7 @@ struct BwdParams {
   float scale_log2;     // scale * log2(e)
   int nblk;             // 128-row blocks per (b, h)
   int units;            // B * H * nblk: one unit = one resident key (dK/dV) or query (dQ) block
+  int out_vec32;        // dq, dk, dv 32-byte aligned: the epilogue writes whole 32-byte sectors
   unsigned long long wait_limit_ns;
 };
 
@@ -169,17 +170,25 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* map, 
 }
 
 // Writes NC (16 or 32) fp32 accumulator columns of one row (times `mul`) as
-// 16-bit values.
+// 16-bit values: 32-byte stores when the row is 32-byte aligned (each fills
+// whole L2 sectors: a 16-byte store from every lane of a warp touches 32 rows
+// with half-sector writes, twice the transactions and a read-modify-write of
+// each sector), else 16-byte stores.
 template <bool BF16, int NC>
-__device__ __forceinline__ void store_acc(void* dst_row, const uint32_t* acc, float mul) {
+__device__ __forceinline__ void store_acc(void* dst_row, const uint32_t* acc, float mul, bool vec32) {
   uint4 w[NC / 8];
   uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
   for (int i = 0; i < NC / 2; ++i)
     wp[i] = pack2<BF16>(__uint_as_float(acc[2 * i]) * mul, __uint_as_float(acc[2 * i + 1]) * mul);
-  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+  if (vec32) {
 #pragma unroll
-  for (int i = 0; i < NC / 8; ++i) dst[i] = w[i];
+    for (int i = 0; i < NC / 16; ++i) st_global_v8(static_cast<uint4*>(dst_row) + 2 * i, wp + 8 * i);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+    for (int i = 0; i < NC / 8; ++i) dst[i] = w[i];
+  }
 }
 
 // One unit of work: a resident key block (dK/dV) or query block (dQ) of one
@@ -560,6 +569,7 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
         const long long row_off = (vec0 + my_row) * HD;
         // this group's quarter of the accumulator columns
         constexpr int EC = HD / (C::COMPUTE_WARPS / 4);
+        const bool vec32 = p.out_vec32 != 0;
         const int c = grp * EC;
         if constexpr (EC == 32) {
           uint32_t a0[32], a1[32];
@@ -567,10 +577,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           if (KV) tmem_ld32_sync(lane_base + C::ACC1_COL + c, a1);
           if (my_row < p.N) {
             if (KV) {
-              store_acc<BF16, 32>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f);
-              store_acc<BF16, 32>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale);
+              store_acc<BF16, 32>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f, vec32);
+              store_acc<BF16, 32>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale, vec32);
             } else {
-              store_acc<BF16, 32>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale);
+              store_acc<BF16, 32>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale, vec32);
             }
           }
         } else {
@@ -580,10 +590,10 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
           if (KV) tmem_ld16_sync(lane_base + C::ACC1_COL + c, a1);
           if (my_row < p.N) {
             if (KV) {
-              store_acc<BF16, 16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f);
-              store_acc<BF16, 16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale);
+              store_acc<BF16, 16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f, vec32);
+              store_acc<BF16, 16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale, vec32);
             } else {
-              store_acc<BF16, 16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale);
+              store_acc<BF16, 16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale, vec32);
             }
           }
         }
