@@ -370,7 +370,9 @@ int launch_bwd_kernel(const BwdParams& p, DeviceState& st, cudaStream_t stream) 
 template <int HD, bool BF16>
 int launch_bwd(const BwdParams& p, DeviceState& st, cudaStream_t stream) {
   const long long rows = (long long)p.B * p.H * p.N;
-  bwd_dsum_kernel<HD, BF16><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p.o, p.dout, p.dsum, rows);
+  constexpr long long kRowsPerBlock = 256 / (HD / 8);  // bwd_dsum_kernel: HD / 8 threads a row
+  bwd_dsum_kernel<HD, BF16><<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, stream>>>(
+      p.o, p.dout, p.dsum, rows);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   int rc = launch_bwd_kernel<HD, BF16, true>(p, st, stream);
   if (rc != FA_OK) return rc;

@@ -14,14 +14,17 @@
 //   dK[j]   = scale * sum_i dS[i,j] Q[i]                 (bwd_dkdv_kernel)
 //   dQ[i]   = scale * sum_j dS[i,j] K[j]                 (bwd_dq_kernel)
 //
-// bwd_dkdv_kernel: one CTA per 128-key block j.  For every query block i it
+// Both kernels run on a persistent grid (min(units, SMs) CTAs taking units in
+// turn); a unit is one resident 128-row block of one (b, h).
+//
+// bwd_dkdv_kernel: a unit per 128-key block j.  For every query block i it
 // computes S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM (tcgen05, SS),
 // forms P^T and dS^T in 16 bits (one thread per key row) and writes them back
 // into TMEM over the dP^T columns it has read, and accumulates
 // dV_j += P^T dO_i and dK_j += dS^T Q_i in TMEM with P^T and dS^T as TMEM
 // operands (tcgen05.mma with A in tensor memory).  The S^T columns are free
 // once read, so S^T for query block i+1 runs during block i's element work.
-// bwd_dq_kernel: one CTA per 128-query block i; recomputes S and dP the same
+// bwd_dq_kernel: a unit per 128-query block i; recomputes S and dP the same
 // way for every key block j and accumulates dQ_i += dS K_j in TMEM.
 // Keeping the 16-bit tiles in TMEM leaves shared memory for five streamed
 // tiles (three of Q / K, two of dO / V), so the blocks after this one load
@@ -132,23 +135,40 @@ struct BwdCfg {
   __host__ __device__ static constexpr uint32_t ds_col(int it, int kk) { return p_col(it, kk) + 16u; }
 };
 
-// D_i = dO_i . O_i in fp32, one warp per row.
+// D_i = dO_i . O_i in fp32: HD / 8 threads per row, each one 16-byte load of
+// O and of dO (8 values), summed across the row's threads by shuffles.
 template <int HD, bool BF16>
 __global__ void __launch_bounds__(256) bwd_dsum_kernel(const void* __restrict__ o,
                                                        const void* __restrict__ dout,
                                                        float* __restrict__ dsum, long long rows) {
-  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
-  const int lane = threadIdx.x % 32;
-  if (row >= rows) return;
-  const T* orow = static_cast<const T*>(o) + row * HD;
-  const T* drow = static_cast<const T*>(dout) + row * HD;
+  using T2 = typename std::conditional<BF16, __nv_bfloat162, __half2>::type;
+  constexpr int TPR = HD / 8;     // threads per row
+  constexpr int RPB = 256 / TPR;  // rows per block
+  const long long row = static_cast<long long>(blockIdx.x) * RPB + threadIdx.x / TPR;
+  const int part = threadIdx.x % TPR;
   float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = *(reinterpret_cast<const uint4*>(o) + row * TPR + part);
+    const uint4 d = *(reinterpret_cast<const uint4*>(dout) + row * TPR + part);
+    const T2* a2 = reinterpret_cast<const T2*>(&a);
+    const T2* d2 = reinterpret_cast<const T2*>(&d);
 #pragma unroll
-  for (int c = lane; c < HD; c += 32) acc += static_cast<float>(orow[c]) * static_cast<float>(drow[c]);
+    for (int i = 0; i < 4; ++i) {
+      float2 x, y;
+      if constexpr (BF16) {
+        x = __bfloat1622float2(a2[i]);
+        y = __bfloat1622float2(d2[i]);
+      } else {
+        x = __half22float2(a2[i]);
+        y = __half22float2(d2[i]);
+      }
+      acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+    }
+  }
+  // every lane takes part in the shuffles; a row's threads are TPR adjacent lanes
 #pragma unroll
-  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-  if (lane == 0) dsum[row] = acc;
+  for (int sh = TPR / 2; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (row < rows && part == 0) dsum[row] = acc;
 }
 
 // Of every 8 argument pairs of P, how many take the FMA-pipe exp2 (exp2_poly2)
