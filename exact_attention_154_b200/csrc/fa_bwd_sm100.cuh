@@ -272,7 +272,8 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
   const int G = gridDim.x, cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
-    // P / dS written: one arrival per compute warp; the rest are single
+    // S read, P written, dS written: one arrival per compute warp; the rest
+    // are single
     for (int i = 0; i < C::NUM_BARS; ++i)
       mbar_init(bars + 8 * i, (i >= C::B_S_READ && i < C::B_DONE) ? C::COMPUTE_WARPS : 1);
     *abort_flag = 0;
@@ -482,145 +483,145 @@ __global__ void __launch_bounds__(BwdCfg<HD, KV>::THREADS, 1)
     bool ok = true;
     int g = 0, k = 0;  // streamed steps and units so far
     for (int round = 0; ok && round * G < p.units; ++round) {
-    const int u = bwd_unit_of(round, cta, G);
-    if (u >= p.units) continue;
-    const BwdUnit w = bwd_unit(p, u, KV);
-    const long long vec0 = static_cast<long long>(w.bh) * p.N;
-    const int my_row = w.blk * 128 + r;  // key row (dkdv) or query row (dq)
-    float my_lse2 = INFINITY, my_dsum = 0.f;
-    if (!KV && my_row < p.N) {
-      my_lse2 = p.lse[vec0 + my_row] * kLog2e;
-      my_dsum = p.dsum[vec0 + my_row];
-    }
-    for (int it = 0; it < w.count; ++it) {
-      const int gs = g + it;
-      const int other0 = (w.first + it) * 128;  // first streamed row of this step
-      // dkdv: the statistics of the streamed query block's columns, lane l
-      // holding column cb + l (+inf lse masks query rows past N); read by
-      // shuffles below
-      float col_lse2 = INFINITY, col_dsum = 0.f;
-      if (KV) {
-        const int qi = other0 + cb + lane;
-        if (qi < p.N) {
-          col_lse2 = p.lse[vec0 + qi] * kLog2e;
-          col_dsum = p.dsum[vec0 + qi];
-        }
+      const int u = bwd_unit_of(round, cta, G);
+      if (u >= p.units) continue;
+      const BwdUnit w = bwd_unit(p, u, KV);
+      const long long vec0 = static_cast<long long>(w.bh) * p.N;
+      const int my_row = w.blk * 128 + r;  // key row (dkdv) or query row (dq)
+      float my_lse2 = INFINITY, my_dsum = 0.f;
+      if (!KV && my_row < p.N) {
+        my_lse2 = p.lse[vec0 + my_row] * kLog2e;
+        my_dsum = p.dsum[vec0 + my_row];
       }
-      ok = wait_phase(bars + 8 * C::B_SD_FULL, gs & 1, abort_flag, lim,
-                      (kRoleSoftmax << 8) | kSiteSFull);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after_sync();
-      // (the 16-bit tiles last written to this step's dP columns were read by
-      // products that the MMA thread issued before this step's dP)
-      // S and dP of this thread's row over the group's 32 columns, one wait
-      uint32_t sd[64];
-      const uint32_t dpc = C::dp_col(gs);
-      tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + dpc + cb, sd);
-      tmem_ld64_wait(sd);
-      // both are in registers: the next S may overwrite the S columns
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * C::B_S_READ);
-      // P (kept in fp32 over the S registers for dS); BWD_POLY8 of every 8
-      // argument pairs take the FMA-pipe exp2, the rest ex2
-      uint32_t pk[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float2 nl = KV ? make_float2(-__shfl_sync(0xffffffffu, col_lse2, 2 * q),
-                                           -__shfl_sync(0xffffffffu, col_lse2, 2 * q + 1))
-                             : make_float2(-my_lse2, -my_lse2);
-        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sd[2 * q]), __uint_as_float(sd[2 * q + 1])),
-                                    make_float2(sl2, sl2), nl);
-        float2 ev;
-        if ((q % 8) >= 8 - BWD_POLY8) {
-          ev = exp2_poly2(x);
-        } else {
-          ev.x = ex2(x.x);
-          ev.y = ex2(x.y);
+      for (int it = 0; it < w.count; ++it) {
+        const int gs = g + it;
+        const int other0 = (w.first + it) * 128;  // first streamed row of this step
+        // dkdv: the statistics of the streamed query block's columns, lane l
+        // holding column cb + l (+inf lse masks query rows past N); read by
+        // shuffles below
+        float col_lse2 = INFINITY, col_dsum = 0.f;
+        if (KV) {
+          const int qi = other0 + cb + lane;
+          if (qi < p.N) {
+            col_lse2 = p.lse[vec0 + qi] * kLog2e;
+            col_dsum = p.dsum[vec0 + qi];
+          }
         }
-        float pp[2] = {ev.x, ev.y};
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = cb + 2 * q + e;
-          // dkdv: row = key my_row, column = query other0 + c (columns past N
-          // carry lse = +inf); dq: row = query my_row, column = key other0 + c
-          const bool vis = KV ? (!p.causal || other0 + c >= my_row)
-                              : (other0 + c < p.N && (!p.causal || other0 + c <= my_row));
-          pp[e] = vis ? pp[e] : 0.f;
-          sd[2 * q + e] = __float_as_uint(pp[e]);
+        ok = wait_phase(bars + 8 * C::B_SD_FULL, gs & 1, abort_flag, lim,
+                        (kRoleSoftmax << 8) | kSiteSFull);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after_sync();
+        // (the 16-bit tiles last written to this step's dP columns were read by
+        // products that the MMA thread issued before this step's dP)
+        // S and dP of this thread's row over the group's 32 columns, one wait
+        uint32_t sd[64];
+        const uint32_t dpc = C::dp_col(gs);
+        tmem_ld32x2_nowait(lane_base + C::S_COL + cb, lane_base + dpc + cb, sd);
+        tmem_ld64_wait(sd);
+        // both are in registers: the next S may overwrite the S columns
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * C::B_S_READ);
+        // P (kept in fp32 over the S registers for dS); BWD_POLY8 of every 8
+        // argument pairs take the FMA-pipe exp2, the rest ex2
+        uint32_t pk[16];
+  #pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float2 nl = KV ? make_float2(-__shfl_sync(0xffffffffu, col_lse2, 2 * q),
+                                             -__shfl_sync(0xffffffffu, col_lse2, 2 * q + 1))
+                               : make_float2(-my_lse2, -my_lse2);
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sd[2 * q]), __uint_as_float(sd[2 * q + 1])),
+                                      make_float2(sl2, sl2), nl);
+          float2 ev;
+          if ((q % 8) >= 8 - BWD_POLY8) {
+            ev = exp2_poly2(x);
+          } else {
+            ev.x = ex2(x.x);
+            ev.y = ex2(x.y);
+          }
+          float pp[2] = {ev.x, ev.y};
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = cb + 2 * q + e;
+            // dkdv: row = key my_row, column = query other0 + c (columns past N
+            // carry lse = +inf); dq: row = query my_row, column = key other0 + c
+            const bool vis = KV ? (!p.causal || other0 + c >= my_row)
+                                : (other0 + c < p.N && (!p.causal || other0 + c <= my_row));
+            pp[e] = vis ? pp[e] : 0.f;
+            sd[2 * q + e] = __float_as_uint(pp[e]);
+          }
+          pk[q] = pack2<BF16>(pp[0], pp[1]);
         }
-        pk[q] = pack2<BF16>(pp[0], pp[1]);
-      }
-      if (KV) {
-        // P^T over the first 16 of the group's dP^T columns (read above)
-        tmem_st16(lane_base + dpc + cb, pk);
+        if (KV) {
+          // P^T over the first 16 of the group's dP^T columns (read above)
+          tmem_st16(lane_base + dpc + cb, pk);
+          tmem_st_wait();
+          tc_fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + (gs & 1)));
+        }
+        // dS = P (dP - D)
+        uint32_t dk[16];
+  #pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float ds[2];
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int c = cb + 2 * q + e;
+            const float pv = __uint_as_float(sd[2 * q + e]);
+            const float dpv = __uint_as_float(sd[32 + 2 * q + e]);
+            ds[e] = pv * (dpv - (KV ? __shfl_sync(0xffffffffu, col_dsum, c - cb) : my_dsum));
+          }
+          dk[q] = pack2<BF16>(ds[0], ds[1]);
+        }
+        // over the last 16 of the group's dP columns
+        tmem_st16(lane_base + dpc + cb + 16, dk);
         tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars + 8 * (C::B_P_FULL + (gs & 1)));
+        if (lane == 0) mbar_arrive(bars + 8 * (C::B_DS_FULL + (gs & 1)));
       }
-      // dS = P (dP - D)
-      uint32_t dk[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        float ds[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = cb + 2 * q + e;
-          const float pv = __uint_as_float(sd[2 * q + e]);
-          const float dpv = __uint_as_float(sd[32 + 2 * q + e]);
-          ds[e] = pv * (dpv - (KV ? __shfl_sync(0xffffffffu, col_dsum, c - cb) : my_dsum));
-        }
-        dk[q] = pack2<BF16>(ds[0], ds[1]);
-      }
-      // over the last 16 of the group's dP columns
-      tmem_st16(lane_base + dpc + cb + 16, dk);
-      tmem_st_wait();
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars + 8 * (C::B_DS_FULL + (gs & 1)));
-    }
-    if (ok) {
-      ok = wait_phase(bars + 8 * C::B_DONE, k & 1, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
-      ok = __all_sync(0xffffffffu, ok);
       if (ok) {
-        tc_fence_after_sync();
-        using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
-        const long long row_off = (vec0 + my_row) * HD;
-        // this group's quarter of the accumulator columns
-        constexpr int EC = HD / (C::COMPUTE_WARPS / 4);
-        const bool vec32 = p.out_vec32 != 0;
-        const int c = grp * EC;
-        if constexpr (EC == 32) {
-          uint32_t a0[32], a1[32];
-          tmem_ld32_sync(lane_base + C::ACC0_COL + c, a0);
-          if (KV) tmem_ld32_sync(lane_base + C::ACC1_COL + c, a1);
-          if (my_row < p.N) {
-            if (KV) {
-              store_acc<BF16, 32>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f, vec32);
-              store_acc<BF16, 32>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale, vec32);
-            } else {
-              store_acc<BF16, 32>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale, vec32);
+        ok = wait_phase(bars + 8 * C::B_DONE, k & 1, abort_flag, lim, (kRoleSoftmax << 8) | kSiteODone);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after_sync();
+          using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+          const long long row_off = (vec0 + my_row) * HD;
+          // this group's quarter of the accumulator columns
+          constexpr int EC = HD / (C::COMPUTE_WARPS / 4);
+          const bool vec32 = p.out_vec32 != 0;
+          const int c = grp * EC;
+          if constexpr (EC == 32) {
+            uint32_t a0[32], a1[32];
+            tmem_ld32_sync(lane_base + C::ACC0_COL + c, a0);
+            if (KV) tmem_ld32_sync(lane_base + C::ACC1_COL + c, a1);
+            if (my_row < p.N) {
+              if (KV) {
+                store_acc<BF16, 32>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f, vec32);
+                store_acc<BF16, 32>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale, vec32);
+              } else {
+                store_acc<BF16, 32>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale, vec32);
+              }
             }
-          }
-        } else {
-          static_assert(EC == 16, "accumulator quarter");
-          uint32_t a0[16], a1[16];
-          tmem_ld16_sync(lane_base + C::ACC0_COL + c, a0);
-          if (KV) tmem_ld16_sync(lane_base + C::ACC1_COL + c, a1);
-          if (my_row < p.N) {
-            if (KV) {
-              store_acc<BF16, 16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f, vec32);
-              store_acc<BF16, 16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale, vec32);
-            } else {
-              store_acc<BF16, 16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale, vec32);
+          } else {
+            static_assert(EC == 16, "accumulator quarter");
+            uint32_t a0[16], a1[16];
+            tmem_ld16_sync(lane_base + C::ACC0_COL + c, a0);
+            if (KV) tmem_ld16_sync(lane_base + C::ACC1_COL + c, a1);
+            if (my_row < p.N) {
+              if (KV) {
+                store_acc<BF16, 16>(static_cast<T*>(p.dv) + row_off + c, a0, 1.f, vec32);
+                store_acc<BF16, 16>(static_cast<T*>(p.dk) + row_off + c, a1, p.scale, vec32);
+              } else {
+                store_acc<BF16, 16>(static_cast<T*>(p.dq) + row_off + c, a0, p.scale, vec32);
+              }
             }
           }
         }
       }
-    }
-    g += w.count;
-    ++k;
+      g += w.count;
+      ++k;
     }
   }
 
