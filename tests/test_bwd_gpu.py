@@ -114,3 +114,14 @@ def test_key_gradients_sum_to_zero():
     torch.cuda.synchronize()
     dkd = dk.double()
     assert dkd.sum(dim=2).abs().max() <= 2e-2 * dkd.abs().sum(dim=2).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_more_units_than_ctas(causal):
+    """160 key blocks and 160 query blocks (B=1, H=40, N=512) on a persistent
+    grid of at most one CTA per SM: some CTAs take a second unit, carrying the
+    ring slots and the per-step barrier phases over from the first."""
+    q, k, v = synth.random_inputs(1, 40, 512, 128, BF16, seed=5200 + int(causal))
+    dout = synth.random_inputs(1, 40, 512, 128, BF16, seed=5300)[0]
+    assert 40 * (512 // 128) > torch.cuda.get_device_properties(0).multi_processor_count
+    _check(q, k, v, dout, causal, BF16, f"B=1 H=40 N=512 causal={causal}")
