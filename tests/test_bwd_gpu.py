@@ -116,12 +116,14 @@ def test_key_gradients_sum_to_zero():
     assert dkd.sum(dim=2).abs().max() <= 2e-2 * dkd.abs().sum(dim=2).max()
 
 
+@pytest.mark.parametrize("d,dtype", [(128, BF16), (64, FP16)])
 @pytest.mark.parametrize("causal", [False, True])
-def test_more_units_than_ctas(causal):
+def test_more_units_than_ctas(causal, d, dtype):
     """160 key blocks and 160 query blocks (B=1, H=40, N=512) on a persistent
     grid of at most one CTA per SM: some CTAs take a second unit, carrying the
-    ring slots and the per-step barrier phases over from the first."""
-    q, k, v = synth.random_inputs(1, 40, 512, 128, BF16, seed=5200 + int(causal))
-    dout = synth.random_inputs(1, 40, 512, 128, BF16, seed=5300)[0]
+    ring slots and the per-step barrier phases over from the first (d = 64:
+    the dK/dV kernel with two dP regions as well)."""
+    q, k, v = synth.random_inputs(1, 40, 512, d, dtype, seed=5200 + int(causal) + d)
+    dout = synth.random_inputs(1, 40, 512, d, dtype, seed=5300 + d)[0]
     assert 40 * (512 // 128) > torch.cuda.get_device_properties(0).multi_processor_count
-    _check(q, k, v, dout, causal, BF16, f"B=1 H=40 N=512 causal={causal}")
+    _check(q, k, v, dout, causal, dtype, f"B=1 H=40 N=512 d={d} causal={causal}")
