@@ -206,7 +206,10 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
  *   d          : 64 or 128 (else FA_ERR_HEADDIM)
  *   scale, causal, dtype, stream: as fa_fwd
  *
- * Asynchronous on `stream`: three kernels (row statistic, dK/dV, dQ).
+ * Asynchronous on `stream`: three kernels (row statistic, dK/dV, dQ); the
+ * last two run on a persistent grid of at most one CTA per SM.  When dq, dk
+ * and dv are all 32-byte aligned their rows are written with 32-byte stores
+ * (whole L2 sectors), else with 16-byte stores; the results are the same.
  * Returns FA_OK or a negative status; FA_ERR_ALIGN if a tensor pointer is not
  * 16-byte aligned or lse / workspace not 4-byte aligned.
  */
