@@ -116,14 +116,15 @@ def test_key_gradients_sum_to_zero():
     assert dkd.sum(dim=2).abs().max() <= 2e-2 * dkd.abs().sum(dim=2).max()
 
 
-@pytest.mark.parametrize("d,dtype", [(128, BF16), (64, FP16)])
+@pytest.mark.parametrize("d,dtype,N", [(128, BF16, 512), (64, FP16, 512), (128, BF16, 500)])
 @pytest.mark.parametrize("causal", [False, True])
-def test_more_units_than_ctas(causal, d, dtype):
-    """160 key blocks and 160 query blocks (B=1, H=40, N=512) on a persistent
-    grid of at most one CTA per SM: some CTAs take a second unit, carrying the
-    ring slots and the per-step barrier phases over from the first (d = 64:
-    the dK/dV kernel with two dP regions as well)."""
-    q, k, v = synth.random_inputs(1, 40, 512, d, dtype, seed=5200 + int(causal) + d)
-    dout = synth.random_inputs(1, 40, 512, d, dtype, seed=5300 + d)[0]
-    assert 40 * (512 // 128) > torch.cuda.get_device_properties(0).multi_processor_count
-    _check(q, k, v, dout, causal, dtype, f"B=1 H=40 N=512 d={d} causal={causal}")
+def test_more_units_than_ctas(causal, d, dtype, N):
+    """160 key blocks and 160 query blocks (B=1, H=40, N=512, or N=500 with a
+    ragged last block) on a persistent grid of at most one CTA per SM: some
+    CTAs take a second unit, carrying the ring slots and the per-step barrier
+    phases over from the first (d = 64: the dK/dV kernel with two dP regions
+    as well)."""
+    q, k, v = synth.random_inputs(1, 40, N, d, dtype, seed=5200 + int(causal) + d + N)
+    dout = synth.random_inputs(1, 40, N, d, dtype, seed=5300 + d + N)[0]
+    assert 40 * ((N + 127) // 128) > torch.cuda.get_device_properties(0).multi_processor_count
+    _check(q, k, v, dout, causal, dtype, f"B=1 H=40 N={N} d={d} causal={causal}")
