@@ -163,7 +163,8 @@ def test_lse_matches_library_logsumexp(oracle_mod, causal):
 
 # The shapes and seed of compare_and_verify in "flash_attention.py"
 # (forceinjection.github.io), (B, N, d) = (1,256,64), (1,512,64), (1,1024,64),
-# (4,512,64) with seed 42, scaled down in N so the pure-NumPy loop stays fast.
+# (4,512,64) with seed 42 (with its 64 x 64 blocks; smaller blocks on smaller
+# shapes, and two ragged shapes, so the pure-NumPy loop stays fast).
 @pytest.mark.parametrize("B,N,d", [(1, 256, 64), (1, 96, 64), (2, 130, 64)])
 @pytest.mark.parametrize("Br,Bc", [(64, 64), (1, 3), (3, 1), (64, 17)])
 @pytest.mark.parametrize("causal", [False, True])
@@ -174,6 +175,17 @@ def test_tiled_recurrence_equals_definition(oracle_mod, B, N, d, Br, Bc, causal)
     q, k, v = (r.standard_normal((B, N, d)) for _ in range(3))
     O, L = oracle_mod.attention(q, k, v, causal=causal)
     Ot, Lt = tiled.flash_forward(q, k, v, causal=causal, Br=Br, Bc=Bc)
+    np.testing.assert_allclose(Ot, O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Lt, L, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("B,N,d", [(1, 512, 64), (1, 1024, 64), (4, 512, 64)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiled_recurrence_on_the_pages_shapes(oracle_mod, B, N, d, causal):
+    r = np.random.default_rng(42)
+    q, k, v = (r.standard_normal((B, N, d)) for _ in range(3))
+    O, L = oracle_mod.attention(q, k, v, causal=causal)
+    Ot, Lt = tiled.flash_forward(q, k, v, causal=causal, Br=64, Bc=64)
     np.testing.assert_allclose(Ot, O, rtol=0, atol=1e-12)
     np.testing.assert_allclose(Lt, L, rtol=0, atol=1e-12)
 
