@@ -10,9 +10,11 @@ Barriers follow the hardware's parity semantics: a wait for parity p passes
 iff (completed phases & 1) != p, so it misreads when the barrier is two
 phases away.  TMA loads and tensor-core products complete after random
 delays.  A run reports deadlock (every role waiting, nothing in flight), any
-wait issued while the barrier was not exactly one phase short of it, and two
-data hazards: O overwritten by a tile's first P V before both softmax groups
-read it, and a ring slot reloaded before its staged O was stored."""
+wait issued while the barrier was not exactly one phase short of it, and
+these data hazards: O overwritten by a tile's first P V before both softmax
+groups read it, a ring slot reloaded before its staged O was stored, a half
+of the shared P buffer overwritten while a P V product still reads it, and a
+P V product reading a P half not written for it."""
 import random, sys
 
 class Bar:
@@ -71,9 +73,12 @@ def next_user(ti, s, j):
     return -1
 
 class Sim:
-    def __init__(s, p, G, cta, seed, shared_full=False):
+    def __init__(s, p, G, cta, seed, shared_full=False, skip_pfree=False):
         # shared_full: one full barrier per slot for K, V and O uses, waited
-        # with the parity of position // ring depth (the first design)
+        # with the parity of position // ring depth (the first design).
+        # skip_pfree: the softmax groups write their half of the shared P
+        # buffer without waiting for its hand-over (a broken protocol, for the
+        # model's own negative test)
         s.p, s.G, s.cta, s.rng = p, G, cta, random.Random(seed)
         s.shared = shared_full
         K = p.KVS
@@ -93,6 +98,10 @@ class Sim:
         s.where = {}; s.ctx = {}
         s.oread = {}; s.prev_tile = {0: None, 1: None}; s.hazards = []; s.slot_state = {}
         s.pend_mma = {}  # thread -> latest completion time
+        s.skip_pfree = skip_pfree
+        # the shared P buffer, by half: (tile, Q tile, block) of the P written
+        # there, and the time the last P V K-steps reading it end
+        s.p_tag = {0: None, 1: None}; s.p_busy = {0: 0, 1: 0}
     def tiles(s):
         r = 0
         while r * s.G < s.p.num_tiles:
@@ -103,7 +112,9 @@ class Sim:
     def later(s, dt, fn): s.events.append((s.now + dt, fn))
     def tma_load(s, bar, nbytes=1):
         s.b[bar].expect(nbytes); s.later(s.rng.randint(1, 40), lambda: s.b[bar].tx_done(nbytes))
-    def mma(s, th): s.pend_mma[th] = max(s.pend_mma.get(th, s.now), s.now) + s.rng.randint(1, 15)
+    def mma(s, th):
+        s.pend_mma[th] = max(s.pend_mma.get(th, s.now), s.now) + s.rng.randint(1, 15)
+        return s.pend_mma[th]
     def commit(s, th, bar):
         t = max(s.pend_mma.get(th, s.now), s.now) + 1
         s.events.append((t, lambda: s.b[bar].arrive()))
@@ -214,7 +225,10 @@ class Sim:
                             if pt is not None and s.oread.get(sx, {}).get(pt, set()) != {0, 1}:
                                 s.hazards.append(('O overwritten before epilogue read', sx, pt, t))
                             s.prev_tile[sx] = t
-                        s.mma('PV'); s.commit('PV', f'PFR{nx}_{half}')
+                        if s.p_tag[half] != (t, sx, j):
+                            s.hazards.append(('P V read a P half not written for it', half, s.p_tag[half], (t, sx, j)))
+                        s.p_busy[half] = max(s.p_busy[half], s.mma('PV'))
+                        s.commit('PV', f'PFR{nx}_{half}')
                     s.commit('PV', f'PVD{sx}'); ppar[0] ^= 1; prod_count += 1
                     if j == ti['hi'][sx] - 1: s.commit('PV', f'OF{sx}')
                 s.commit('PV', f'KE{v % K}')
@@ -254,7 +268,7 @@ class Sim:
                 yield from meet()
                 s.b[f'SFR{sx}'].arrive(4)
                 rescale = j > lo and s.rng.random() < 0.2
-                if not first_use:
+                if not first_use and not s.skip_pfree:
                     s.check_alias(f'PFR{sx}_{hf}', pfree_seen, who)
                     yield from s.wait(f'PFR{sx}_{hf}', pfpar, who); pfpar ^= 1; pfree_seen += 1
                 first_use = False
@@ -265,6 +279,10 @@ class Sim:
                     s.otouch(sx, hf, 'rescale', t)
                 if hf == 1: s.b['PF0'].arrive(4)
                 yield ('work',)
+                # this group's half of P: the previous user's K-steps must have ended
+                if s.now < s.p_busy[hf]:
+                    s.hazards.append(('P half overwritten while P V reads it', hf, (t, sx, j)))
+                s.p_tag[hf] = (t, sx, j)
                 s.b[f'PF{hf}'].arrive(4)
                 pv_count += 1
             s.check_alias(f'OF{sx}', fin_seen, who)

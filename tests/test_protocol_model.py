@@ -7,8 +7,9 @@ several work tiles.  Random completion times, several seeds each.
 
 Each run must finish without deadlock, without a wait that a parity test
 could misread (barrier not exactly one phase short), without O being
-overwritten before the epilogue read it, and without a ring slot being
-reloaded before its staged O was stored."""
+overwritten before the epilogue read it, without a ring slot being reloaded
+before its staged O was stored, and with every P V product reading the P
+half written for it, never overwritten while it reads."""
 import pytest
 
 import protocol_model as pm
@@ -50,4 +51,18 @@ def test_model_flags_a_shared_full_barrier():
             sim = pm.Sim(p, 148, cta, seed, shared_full=True)
             r = sim.run(max_steps=400000)
             bad += (r != "ok") or bool(sim.aliased) or bool(sim.hazards)
+    assert bad > 0
+
+
+def test_model_flags_a_p_half_written_before_its_hand_over():
+    """The model checks the shared P buffer's data too: softmax groups that
+    write their half without waiting for the previous user's P V K-steps to
+    end overwrite P that a product still reads, in some schedule."""
+    p = pm.P(N=2048, causal=False, QS=2, KVS=4, B=1, H=2)
+    bad = 0
+    for cta in (0, 1):
+        for seed in range(3):
+            sim = pm.Sim(p, 2, cta, seed, skip_pfree=True)
+            r = sim.run(max_steps=400000)
+            bad += (r != "ok") or bool(sim.hazards)
     assert bad > 0
