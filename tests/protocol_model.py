@@ -12,9 +12,12 @@ phases away.  TMA loads and tensor-core products complete after random
 delays.  A run reports deadlock (every role waiting, nothing in flight), any
 wait issued while the barrier was not exactly one phase short of it, and
 these data hazards: O overwritten by a tile's first P V before both softmax
-groups read it, a ring slot reloaded before its staged O was stored, a half
-of the shared P buffer overwritten while a P V product still reads it, and a
-P V product reading a P half not written for it."""
+groups read it, a ring slot reloaded before its staged O was stored or while
+an MMA still reads it, an S or P V product reading a slot that does not hold
+its own K or V, a softmax group reading an S buffer that does not hold its
+block's scores, a half of the shared P buffer overwritten while a P V
+product still reads it, and a P V product reading a P half not written for
+it."""
 import random, sys
 
 class Bar:
@@ -73,12 +76,14 @@ def next_user(ti, s, j):
     return -1
 
 class Sim:
-    def __init__(s, p, G, cta, seed, shared_full=False, skip_pfree=False):
+    def __init__(s, p, G, cta, seed, shared_full=False, skip_pfree=False, skip_sfree=False):
         # shared_full: one full barrier per slot for K, V and O uses, waited
         # with the parity of position // ring depth (the first design).
         # skip_pfree: the softmax groups write their half of the shared P
         # buffer without waiting for its hand-over (a broken protocol, for the
-        # model's own negative test)
+        # model's own negative test).  skip_sfree: the S thread overwrites a
+        # Q tile's S buffer without waiting for the softmax to have read it
+        # (likewise broken)
         s.p, s.G, s.cta, s.rng = p, G, cta, random.Random(seed)
         s.shared = shared_full
         K = p.KVS
@@ -102,6 +107,10 @@ class Sim:
         # the shared P buffer, by half: (tile, Q tile, block) of the P written
         # there, and the time the last P V K-steps reading it end
         s.p_tag = {0: None, 1: None}; s.p_busy = {0: 0, 1: 0}
+        s.skip_sfree = skip_sfree
+        # ring slots: the (tile, 'K' / 'V', block) last landed there and the
+        # time its last reader ends; S buffers: the (tile, block) of the S in it
+        s.slot_data = {}; s.slot_busy = {}; s.s_tag = {0: None, 1: None}
     def tiles(s):
         r = 0
         while r * s.G < s.p.num_tiles:
@@ -134,14 +143,22 @@ class Sim:
     def producer(s):
         p, K = s.p, s.p.KVS
         kv = [0]; q_count = 0
-        def load_kv(tag):
+        def load_kv(tag, ident):
             slot, use = kv[0] % K, kv[0] // K
             if use > 0:
                 s.check_alias(f'KE{slot}', use - 1, 'prod')
                 yield from s.wait(f'KE{slot}', (use - 1) & 1, 'prod')
             if s.slot_state.get(slot, ('',))[0] == 'O-staged': s.hazards.append(('slot reloaded before O store', slot))
+            if s.now < s.slot_busy.get(slot, 0):
+                s.hazards.append(('slot reloaded while an MMA reads it', slot, ident))
             s.slot_state[slot] = ('KV',)
-            s.tma_load(('KF' if s.shared else ('KS' if tag == 'K' else 'KV')) + str(slot)); kv[0] += 1
+            bar = ('KF' if s.shared else ('KS' if tag == 'K' else 'KV')) + str(slot)
+            s.b[bar].expect(1)
+
+            def land(slot=slot, ident=ident, bar=bar):
+                s.slot_data[slot] = ident
+                s.b[bar].tx_done(1)
+            s.later(s.rng.randint(1, 40), land); kv[0] += 1
         def reserve():
             slot, use = kv[0] % K, kv[0] // K
             if use > 0:
@@ -151,15 +168,16 @@ class Sim:
         for t in s.tiles():
             ti = decode(p, t)
             if ti['n_u'] == 0: continue
-            yield from load_kv('K')
+            yield from load_kv('K', (t, 'K', ti['lo_u']))
             if q_count > 0:
                 s.check_alias('QE', q_count - 1, 'prod')
                 yield from s.wait('QE', (q_count - 1) & 1, 'prod')
             s.tma_load('QF'); q_count += 1
             for jj in range(ti['n_u']):
                 s.ctx['prod'] = ('tile', t, 'jj', jj, 'kv', kv[0])
-                if jj + 1 < ti['n_u']: yield from load_kv('K')
-                yield from load_kv('V')
+                j = ti['lo_u'] + jj
+                if jj + 1 < ti['n_u']: yield from load_kv('K', (t, 'K', j + 1))
+                yield from load_kv('V', (t, 'V', j))
             for sx in range(p.QS):
                 s.ctx['prod'] = ('tile', t, 'reserve', sx, 'kv', kv[0])
                 if via_slot(p, ti, sx): yield from reserve()
@@ -187,10 +205,15 @@ class Sim:
                 yield from wait_kv(k)
                 for sx in range(p.QS):
                     if inr(ti, sx, j):
-                        if issued[sx] > 0:
+                        if issued[sx] > 0 and not s.skip_sfree:
                             s.check_alias(f'SFR{sx}', issued[sx] - 1, 'S')
                             yield from s.wait(f'SFR{sx}', sf[sx], 'S'); sf[sx] ^= 1
-                        s.mma('S'); s.commit('S', f'SF{sx}'); issued[sx] += 1
+                        if s.slot_data.get(k % K) != (t, 'K', j):
+                            s.hazards.append(('S read a slot not holding its K', k % K, s.slot_data.get(k % K), (t, 'K', j)))
+                        end = s.mma('S')
+                        s.slot_busy[k % K] = max(s.slot_busy.get(k % K, 0), end)
+                        s.events.append((end, lambda sx=sx, tag=(t, j): s.s_tag.__setitem__(sx, tag)))
+                        s.commit('S', f'SF{sx}'); issued[sx] += 1
                 s.commit('S', f'KE{k % K}')
                 if jj + 1 == ti['n_u']: s.commit('S', 'QE')
             kv = kv0 + 2 * ti['n_u'] + nslots(p, ti)
@@ -213,6 +236,8 @@ class Sim:
                 else:
                     s.check_alias(f'KV{sl}', vuse[sl], 'PV')
                     yield from s.wait(f'KV{sl}', vuse[sl] & 1, 'PV'); vuse[sl] += 1
+                if s.slot_data.get(sl) != (t, 'V', j):
+                    s.hazards.append(('P V read a slot not holding its V', sl, s.slot_data.get(sl), (t, 'V', j)))
                 for sx in range(p.QS):
                     if not inr(ti, sx, j): continue
                     nx = next_user(ti, sx, j); nx = 0 if nx < 0 else nx
@@ -227,7 +252,9 @@ class Sim:
                             s.prev_tile[sx] = t
                         if s.p_tag[half] != (t, sx, j):
                             s.hazards.append(('P V read a P half not written for it', half, s.p_tag[half], (t, sx, j)))
-                        s.p_busy[half] = max(s.p_busy[half], s.mma('PV'))
+                        end = s.mma('PV')
+                        s.p_busy[half] = max(s.p_busy[half], end)
+                        s.slot_busy[sl] = max(s.slot_busy.get(sl, 0), end)
                         s.commit('PV', f'PFR{nx}_{half}')
                     s.commit('PV', f'PVD{sx}'); ppar[0] ^= 1; prod_count += 1
                     if j == ti['hi'][sx] - 1: s.commit('PV', f'OF{sx}')
@@ -264,6 +291,8 @@ class Sim:
                 s.ctx[who] = ('tile', t, 'j', j)
                 s.check_alias(f'SF{sx}', s_seen, who)
                 yield from s.wait(f'SF{sx}', spar, who); spar ^= 1; s_seen += 1
+                if s.s_tag[sx] != (t, j):
+                    s.hazards.append(('softmax read an S not computed for it', sx, s.s_tag[sx], (t, j)))
                 yield ('work',)
                 yield from meet()
                 s.b[f'SFR{sx}'].arrive(4)

@@ -66,3 +66,17 @@ def test_model_flags_a_p_half_written_before_its_hand_over():
             r = sim.run(max_steps=400000)
             bad += (r != "ok") or bool(sim.hazards)
     assert bad > 0
+
+
+def test_model_flags_an_s_buffer_overwritten_before_it_was_read():
+    """Likewise for the S buffers: an S thread that issues S(j+1) of a Q tile
+    without waiting for its softmax to have read S(j) hands the softmax the
+    wrong block's scores in some schedule."""
+    p = pm.P(N=2048, causal=False, QS=2, KVS=4, B=1, H=2)
+    bad = 0
+    for cta in (0, 1):
+        for seed in range(3):
+            sim = pm.Sim(p, 2, cta, seed, skip_sfree=True)
+            r = sim.run(max_steps=400000)
+            bad += (r != "ok") or bool(sim.hazards)
+    assert bad > 0
