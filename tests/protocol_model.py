@@ -13,8 +13,9 @@ delays.  A run reports deadlock (every role waiting, nothing in flight), any
 wait issued while the barrier was not exactly one phase short of it, and
 these data hazards: O overwritten by a tile's first P V before both softmax
 groups read it, a ring slot reloaded before its staged O was stored or while
-an MMA still reads it, an S or P V product reading a slot that does not hold
-its own K or V, a softmax group reading an S buffer that does not hold its
+an MMA still reads it, the Q buffer reloaded while an S product reads it, an
+S or P V product reading a Q buffer or slot that does not hold its own Q, K
+or V, a softmax group reading an S buffer that does not hold its
 block's scores, a half of the shared P buffer overwritten while a P V
 product still reads it, and a P V product reading a P half not written for
 it."""
@@ -76,14 +77,16 @@ def next_user(ti, s, j):
     return -1
 
 class Sim:
-    def __init__(s, p, G, cta, seed, shared_full=False, skip_pfree=False, skip_sfree=False):
+    def __init__(s, p, G, cta, seed, shared_full=False, skip_pfree=False, skip_sfree=False,
+                 skip_qempty=False):
         # shared_full: one full barrier per slot for K, V and O uses, waited
         # with the parity of position // ring depth (the first design).
         # skip_pfree: the softmax groups write their half of the shared P
         # buffer without waiting for its hand-over (a broken protocol, for the
         # model's own negative test).  skip_sfree: the S thread overwrites a
         # Q tile's S buffer without waiting for the softmax to have read it
-        # (likewise broken)
+        # (likewise broken).  skip_qempty: the producer loads the next work
+        # tile's Q without waiting for the last S product of this one
         s.p, s.G, s.cta, s.rng = p, G, cta, random.Random(seed)
         s.shared = shared_full
         K = p.KVS
@@ -111,6 +114,10 @@ class Sim:
         # ring slots: the (tile, 'K' / 'V', block) last landed there and the
         # time its last reader ends; S buffers: the (tile, block) of the S in it
         s.slot_data = {}; s.slot_busy = {}; s.s_tag = {0: None, 1: None}
+        s.skip_qempty = skip_qempty
+        # the Q buffer: the work tile whose Q landed there, and the time its
+        # last S product ends
+        s.q_data = None; s.q_busy = 0
     def tiles(s):
         r = 0
         while r * s.G < s.p.num_tiles:
@@ -169,10 +176,17 @@ class Sim:
             ti = decode(p, t)
             if ti['n_u'] == 0: continue
             yield from load_kv('K', (t, 'K', ti['lo_u']))
-            if q_count > 0:
+            if q_count > 0 and not s.skip_qempty:
                 s.check_alias('QE', q_count - 1, 'prod')
                 yield from s.wait('QE', (q_count - 1) & 1, 'prod')
-            s.tma_load('QF'); q_count += 1
+            if s.now < s.q_busy:
+                s.hazards.append(('Q reloaded while an S product reads it', t))
+            s.b['QF'].expect(1)
+
+            def land_q(t=t):
+                s.q_data = t
+                s.b['QF'].tx_done(1)
+            s.later(s.rng.randint(1, 40), land_q); q_count += 1
             for jj in range(ti['n_u']):
                 s.ctx['prod'] = ('tile', t, 'jj', jj, 'kv', kv[0])
                 j = ti['lo_u'] + jj
@@ -208,10 +222,13 @@ class Sim:
                         if issued[sx] > 0 and not s.skip_sfree:
                             s.check_alias(f'SFR{sx}', issued[sx] - 1, 'S')
                             yield from s.wait(f'SFR{sx}', sf[sx], 'S'); sf[sx] ^= 1
+                        if s.q_data != t:
+                            s.hazards.append(('S read a Q buffer not holding its tile', s.q_data, t))
                         if s.slot_data.get(k % K) != (t, 'K', j):
                             s.hazards.append(('S read a slot not holding its K', k % K, s.slot_data.get(k % K), (t, 'K', j)))
                         end = s.mma('S')
                         s.slot_busy[k % K] = max(s.slot_busy.get(k % K, 0), end)
+                        s.q_busy = max(s.q_busy, end)
                         s.events.append((end, lambda sx=sx, tag=(t, j): s.s_tag.__setitem__(sx, tag)))
                         s.commit('S', f'SF{sx}'); issued[sx] += 1
                 s.commit('S', f'KE{k % K}')

@@ -80,3 +80,18 @@ def test_model_flags_an_s_buffer_overwritten_before_it_was_read():
             r = sim.run(max_steps=400000)
             bad += (r != "ok") or bool(sim.hazards)
     assert bad > 0
+
+
+def test_model_flags_a_q_buffer_reloaded_too_early():
+    """And for the Q buffer: loading the next work tile's Q without waiting
+    for this tile's last S product shows an S reading the wrong Q in some
+    schedule."""
+    # a deep ring (d = 64) lets the producer run a work tile ahead
+    p = pm.P(N=512, causal=False, QS=2, KVS=10, B=2, H=8)
+    bad = 0
+    for cta in (0, 1):
+        for seed in range(3):
+            sim = pm.Sim(p, 2, cta, seed, skip_qempty=True)
+            r = sim.run(max_steps=400000)
+            bad += (r != "ok") or bool(sim.hazards)
+    assert bad > 0
