@@ -1,6 +1,6 @@
 """The forward kernel's mbarrier protocol, run in a CPU model
 (``tests/protocol_model.py``) over schedules that cover every kernel
-configuration: the three ring depths (2, 4 and 10 slots), one and two Q
+configuration: the ring depths (2, 4, 5 and 10 slots), one and two Q
 tiles per work tile, causal and non-causal, a local window, packed
 variable-length sequences with empty and partial tiles, and CTAs with one or
 several work tiles.  Random completion times, several seeds each.
@@ -23,6 +23,9 @@ CASES = [
     dict(N=1024, causal=True, QS=2, KVS=4, B=2, H=2, left=100),
     dict(N=600, causal=True, QS=2, KVS=4, lens=[1, 7, 128, 0, 129, 300, 513, 256], H=3),
     dict(N=1000, causal=False, QS=2, KVS=10, B=1, H=2, left=64, right=3),
+    # e4m3: d = 128 with a 10-slot ring, d = 256 with 5 slots; O by direct stores
+    dict(N=2048, causal=False, QS=2, KVS=10, B=2, H=4, o_tma=False),
+    dict(N=4096, causal=True, QS=1, KVS=5, B=1, H=4, o_tma=False),
 ]
 
 
