@@ -19,7 +19,7 @@ or V, a softmax group reading an S buffer that does not hold its
 block's scores, a half of the shared P buffer overwritten while a P V
 product still reads it, and a P V product reading a P half not written for
 it."""
-import random, sys
+import random
 
 class Bar:
     def __init__(s, name, count): s.name, s.count, s.pending, s.tx, s.c = name, count, count, 0, 0

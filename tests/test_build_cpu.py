@@ -1,6 +1,5 @@
 """Host-only checks of the build inputs, the binding's device checks and the
 software exp2's coefficients.  No GPU."""
-import math
 import os
 import re
 

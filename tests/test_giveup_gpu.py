@@ -9,7 +9,6 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 from exact_attention_154_b200 import fa, synth
 from exact_attention_154_b200.synth import BF16
 

@@ -15,7 +15,6 @@ decoded as normal, descale_v applied to the scores, and descale_k dropped
 each break a pin.
 """
 import numpy as np
-import pytest
 import torch
 
 import oracle
