@@ -44,3 +44,42 @@ def imbalance(N, B, H, causal, QS=2):
 ])
 def test_longest_first_snake_balances_the_work(N, B, H, causal, QS, bound):
     assert imbalance(N, B, H, causal, QS) <= bound
+
+
+def bwd_imbalance(B, H, N, causal, kv):
+    """The backward kernels' persistent hand-out, restated: units in (b, h)
+    order (non-causal) or longest first (causal: key block 0 of every head for
+    dK/dV, the last query block for dQ), snake over min(units, SMs) CTAs;
+    work = streamed blocks per unit."""
+    nblk = (N + 127) // 128
+    units = B * H * nblk
+    G = min(SMS, units)
+
+    def blocks(u):
+        if causal:
+            rank = u // (B * H)
+            blk = rank if kv else nblk - 1 - rank
+        else:
+            blk = u % nblk
+        first = blk if (kv and causal) else 0
+        last = blk if (not kv and causal) else nblk - 1
+        return last - first + 1
+
+    work = [0] * G
+    r = 0
+    while r * G < units:
+        for c in range(G):
+            u = r * G + ((G - 1 - c) if r & 1 else c)
+            if u < units:
+                work[c] += blocks(u)
+        r += 1
+    assert sum(work) == B * H * (nblk * (nblk + 1) // 2 if causal else nblk * nblk)
+    return max(work) * G / sum(work)
+
+
+@pytest.mark.parametrize("B,H,N,causal", [(4, 16, 4096, False), (4, 16, 4096, True),
+                                           (16, 16, 1024, False), (16, 16, 1024, True),
+                                           (1, 16, 16384, True)])
+@pytest.mark.parametrize("kv", [True, False])
+def test_backward_hand_out_balances_the_work(B, H, N, causal, kv):
+    assert bwd_imbalance(B, H, N, causal, kv) <= 1.015
