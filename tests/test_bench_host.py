@@ -79,3 +79,11 @@ def test_peak_follows_the_length_of_the_timed_region():
     assert p == 2 * 1662.1 and "x 2" in note
     p, _ = bench.pick_peak(dict(bench.FALLBACK_PEAKS), "fallback", 2.0)
     assert p == bench.FALLBACK_PEAKS["bf16_tflops_sustained"]
+
+
+def test_committed_traffic_record_matches_the_current_sources():
+    """The committed ncu traffic record was taken on the sources in the tree:
+    bench.py reports it for the profiled workloads (after a kernel change the
+    record must be re-taken, or this fails)."""
+    for key in ("sweep-n4096", "causal-h128-n2048", "hd256-causal-n8192", "bwd:sweep-n4096"):
+        assert bench.profiled_traffic(key) is not None, key
